@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the exact IO-aware attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole bf16 path over one batch: fa_fwd (O, LSE)
+followed by fa_bwd (preprocess, recompute kernel, dQ finalize).  The workload
+is the B=4, H=16, N=2048, d=64 non-causal bf16 attention with Q, K, V, dO ~
+N(0, 1) (seeded synthetic inputs).  The metric is attention TFLOP/s:
+  forward FLOPs F = 4 B H N^2 d (halved when causal), backward 2.5 F,
+  fwd+bwd TFLOP/s = 3.5 F / (t_fwd + t_bwd).
+Rank 0 prints ONE JSON line.  Under torchrun every rank runs its own batch
+(weak scaling, no collective on the data path); `value` is the FLOPs of all
+ranks divided by the slowest rank's time.
+
+`--impl reference` times the fp64 CPU oracle (the correctness reference) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(B=4, H=16, N=2048, d=64, causal=False)
+WORKLOAD_NAME = "attention fwd+bwd bf16 B4 H16 N2048 d64 non-causal"
+METRIC = "attention TFLOP/s fwd & fwd+bwd (bf16) and % of B200 dense tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def fwd_flops(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d
+    return f / 2.0 if causal else f
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and clock-event reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [x for x in sm if smax and x > 0.3 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# -------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+
+    import exact_io_aware_55_b200 as fa
+    import synth
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    B, H, N, d, causal = (WORKLOAD[k] for k in ("B", "H", "N", "d", "causal"))
+    scale = 1.0 / math.sqrt(d)
+    seed = 4242 + rank
+    inp = synth.attention_inputs(B, H, N, d, seed=seed, want_f64=False)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v, do = (to_dev(inp[n + "_bits"]) for n in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsz = fa.fa_bwd_workspace_size(B, H, N, d)
+    work = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fa_fwd(q, k, v, o, lse, scale, causal, stream)
+        fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale, causal, work, stream)
+
+    F = fwd_flops(B, H, N, d, causal)
+
+    def timed(K, W, sampler_window_s=1.5):
+        for _ in range(W):
+            flush.fill_(1.0)
+            step()
+        torch.cuda.synchronize()
+        # keep the GPU busy for a clock window so the sampler sees the loaded clock
+        sampler = ClockSampler(local)
+        sampler.start()
+        t_end = time.time() + sampler_window_s
+        while time.time() < t_end:
+            for _ in range(20):
+                flush.fill_(1.0)
+                step()
+            torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.fill_(1.0)                     # L2 flush, outside the events
+            ev[i][0].record(stream)
+            fa.fa_fwd(q, k, v, o, lse, scale, causal, stream)
+            ev[i][1].record(stream)
+            fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale, causal, work, stream)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        clocks = sampler.stop()
+        t_fwd = sum(a.elapsed_time(b) for a, b, _ in ev) / K
+        t_bwd = sum(b.elapsed_time(c) for _, b, c in ev) / K
+        return t_fwd, t_bwd, clocks
+
+    t_fwd, t_bwd, clocks = timed(args.steps, args.warmup)
+    if any(r in clocks["reasons"] for r in BAD_REASONS):
+        t_fwd, t_bwd, clocks = timed(args.steps, args.warmup)   # re-measure once
+        clocks["remeasured"] = True
+    st, where = fa.fa_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} (wait site {where}) during the bench")
+
+    t_step = t_fwd + t_bwd
+    if dist is not None:
+        tt = torch.tensor([t_step, t_fwd, t_bwd], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step, t_fwd, t_bwd = (float(x) for x in tt.tolist())
+    value = ws * 3.5 * F / (t_step * 1e-3) / 1e12
+    fwd_tflops = ws * F / (t_fwd * 1e-3) / 1e12
+    bwd_tflops = ws * 2.5 * F / (t_bwd * 1e-3) / 1e12
+
+    # ---------------- e2e through the public API with pinned host buffers
+    host = {n: torch.from_numpy(np.ascontiguousarray(inp[n + "_bits"]).view(np.int16)).view(torch.bfloat16)
+            .pin_memory() for n in ("q", "k", "v", "do")}
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+
+    def e2e_step():
+        qd = host["q"].to(dev, non_blocking=True)
+        kd = host["k"].to(dev, non_blocking=True)
+        vd = host["v"].to(dev, non_blocking=True)
+        dod = host["do"].to(dev, non_blocking=True)
+        od, lsed = fa.attention_forward(qd, kd, vd, scale=scale, causal=causal)
+        gq, gk, gv = fa.attention_backward(qd, kd, vd, od, dod, lsed, scale=scale, causal=causal, workspace=work)
+        for n, t in (("o", od), ("lse", lsed), ("dq", gq), ("dk", gk), ("dv", gv)):
+            host_out[n].copy_(t, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    K2 = max(5, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(K2):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1) / K2
+    if dist is not None:
+        tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_e2e = float(tt.item())
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    # ---------------- extra measurements (rank 0, not part of `value`)
+    extra = {}
+    if rank == 0 and not args.no_extra:
+        extra = extra_measurements(fa, torch, synth, dev, stream)
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    roof = {"bound": "tensor", "kernel": "fa_bwd (bwd_kernel + its preprocess and dQ-finalize launches)",
+            "achieved": round(bwd_tflops / ws, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(bwd_tflops / ws / peak, 4), "traffic": committed_traffic("bwd_kernel", WORKLOAD_NAME),
+            "peak_source": f"{peak_src} bf16_tflops (burst; each launch is timed alone)"}
+
+    if rank == 0:
+        cpu = cpu_baseline(args) if ws >= 1 and not args.no_cpu_baseline and ws == 1 else None
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Philox, rounded to bf16)",
+            "config": {"workload": WORKLOAD_NAME, "B": B, "H": H, "N": N, "d": d, "causal": causal,
+                       "global_batch": B * ws, "seq_len": N, "parallelism": f"dp{ws} (independent batches)",
+                       "l2": "256 MiB flush write between steps, outside the per-step CUDA events"},
+            "fwd_tflops": round(fwd_tflops, 2), "bwd_tflops": round(bwd_tflops, 2),
+            "fwd_frac_of_peak": round(fwd_tflops / ws / peak, 4),
+            "fwd_bwd_frac_of_peak": round(value / ws / peak, 4),
+            "ms_fwd": round(t_fwd, 5), "ms_bwd": round(t_bwd, 5),
+            "e2e": {"value": round(ws * 3.5 * F / (t_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "ms_per_step": round(t_e2e, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "roofline": roof,
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
+            "cpu_baseline": cpu,
+            "extra": extra,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the library build that is loaded now (same source digest); else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    digest_path = os.path.join(ROOT, "exact_io_aware_55_b200", "libfa.so.sha256")
+    if not (os.path.exists(path) and os.path.exists(digest_path)):
+        return None
+    try:
+        data = json.load(open(path))
+        digest = open(digest_path).read().strip()
+        ent = data.get(kernel, {})
+        if ent.get("source_digest") == digest and ent.get("workload") == workload:
+            return ent.get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+    return None
+
+
+def extra_measurements(fa, torch, synth, dev, stream):
+    """Single-GPU context numbers: long-sequence non-causal bf16 (fwd and bwd at
+    N=8192, d=128) and the e4m3 forward at B2 H16 N16384 d128."""
+    out = {}
+
+    def time_call(fn, iters=10, warm=3):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    peaks, _ = load_peaks()
+    B, H, N, d = 1, 32, 8192, 128
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    q, k, v, do = (torch.randn((B, H, N, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+                   for _ in range(4))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    work = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    sc = 1.0 / math.sqrt(d)
+    F = fwd_flops(B, H, N, d, False)
+    tf = time_call(lambda: fa.fa_fwd(q, k, v, o, lse, sc, False, stream))
+    tb = time_call(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, sc, False, work, stream))
+    out["noncausal_b1_h32_n8192_d128"] = {
+        "fwd_tflops": round(F / tf / 1e9, 1), "fwd_frac": round(F / tf / 1e9 / peaks["bf16_tflops"], 4),
+        "bwd_tflops": round(2.5 * F / tb / 1e9, 1), "bwd_frac": round(2.5 * F / tb / 1e9 / peaks["bf16_tflops"], 4),
+        "inputs": "N(0,1) from torch's seeded CUDA generator (timing only)"}
+    del q, k, v, do, o, dq, dk, dv, work
+    B, H, N, d = 2, 16, 16384, 128
+    q8, k8, v8 = (torch.randn((B, H, N, d), generator=g, device=dev).mul_(100.0).clamp_(-448, 448)
+                  .to(torch.float8_e4m3fn) for _ in range(3))
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), device=dev)
+    F = fwd_flops(B, H, N, d, False)
+    try:
+        t8 = time_call(lambda: fa.fa_fwd_fp8(q8, k8, v8, 0.01, 0.01, 0.01, o, lse, 1.0 / math.sqrt(d), False, stream))
+        fp8_peak = 2.0 * peaks["bf16_tflops"]
+        out["fp8_fwd_b2_h16_n16384_d128"] = {
+            "tflops": round(F / t8 / 1e9, 1), "frac_of_fp8_peak": round(F / t8 / 1e9 / fp8_peak, 4),
+            "fp8_peak": fp8_peak, "fp8_peak_source": "2 x measured bf16 (nominal fp8:bf16 dense ratio)"}
+    except Exception as e:  # noqa: BLE001
+        out["fp8_fwd_b2_h16_n16384_d128"] = {"error": str(e)}
+    return out
+
+
+# ------------------------------------------------------------- CPU oracle
+def _oracle_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((x.get("num_threads") or 1) for x in info if x.get("user_api") == "blas")
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def oracle_sample(budget_s: float, seed: int = 4242):
+    """fwd+bwd of whole heads of the bench workload with the fp64 oracle until
+    the time budget is spent.  Returns (TFLOP/s, heads, seconds)."""
+    import oracle
+    import synth
+
+    B, H, N, d, causal = (WORKLOAD[k] for k in ("B", "H", "N", "d", "causal"))
+    inp = synth.attention_inputs(1, 4, N, d, seed=seed, want_f64=False)
+    scale = 1.0 / math.sqrt(d)
+    heads, t0 = 0, time.perf_counter()
+    while True:
+        h = heads % 4
+        qh, kh, vh, doh = (synth.head_f64(inp, n, 0, h) for n in ("q", "k", "v", "do"))
+        oracle.head_backward(qh, kh, vh, doh, scale, causal)     # includes the forward
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or heads >= B * H:
+            break
+    flops = 3.5 * fwd_flops(1, 1, N, d, causal) * heads
+    return flops / el / 1e12, heads, el
+
+
+def cpu_baseline(args):
+    tflops, heads, el = oracle_sample(args.cpu_budget)
+    return {"value": tflops, "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"{heads} of the 64 heads (fwd+bwd, fp64 numpy/OpenBLAS) of the bench workload in {el:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    per_step, heads_total, t_total = [], 0, 0.0
+    for _ in range(args.warmup):
+        oracle_sample(0.0)
+    for _ in range(args.steps):
+        tf, heads, el = oracle_sample(args.ref_step_budget)
+        per_step.append(el)
+        heads_total += heads
+        t_total += el
+    F = 3.5 * fwd_flops(1, 1, WORKLOAD["N"], WORKLOAD["d"], WORKLOAD["causal"]) * heads_total
+    value = F / t_total / 1e12
+    cores = _oracle_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) Philox, rounded to bf16, evaluated in fp64)",
+        "config": {"workload": WORKLOAD_NAME, **WORKLOAD},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: whole heads (fwd+bwd) for {args.ref_step_budget:.1f} s; "
+                                   f"{heads_total} heads in total"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-step-budget", type=float, default=1.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,131 @@
+"""Exact IO-aware attention for B200 (sm_100a).
+
+The compute lives in ``libfa.so`` (C ABI, ``include/fa.h``); this package is
+its Python binding.  Functions named like the C entry points take torch CUDA
+tensors and pass their pointers through unchanged; PyTorch only provides the
+device memory and the stream.  ``attention_forward`` / ``attention_backward``
+additionally allocate the outputs (and the backward workspace) with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import FA_OK, FAError, LIB_PATH, STATUS_CODES, STATUS_NAMES, check, lib, strerror
+
+__all__ = [
+    "FAError", "LIB_PATH", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_size", "fa_device_status",
+    "fa_watchdog_selftest", "attention_forward", "attention_backward", "attention_forward_fp8", "lib",
+    "STATUS_NAMES", "STATUS_CODES", "strerror",
+]
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("tensors must be [B, H, N, d]")
+    return tuple(int(x) for x in q.shape)
+
+
+def _check_tensors(ref_shape, dtype, *ts):
+    for t in ts:
+        if t.device.type != "cuda":
+            raise ValueError("tensors must be CUDA tensors")
+        if tuple(t.shape) != ref_shape or t.dtype != dtype or not t.is_contiguous():
+            raise ValueError(f"expected contiguous {dtype} {ref_shape}, got {t.dtype} {tuple(t.shape)}")
+
+
+def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
+    """O, LSE <- attention(q, k, v) (bf16 in/out, LSE fp32 [B,H,N])."""
+    B, H, N, d = _shape(q)
+    _check_tensors((B, H, N, d), torch.bfloat16, q, k, v, o)
+    _check_tensors((B, H, N), torch.float32, lse)
+    check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale), int(bool(causal)),
+                     _stream_ptr(stream)))
+
+
+def fa_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, o, lse, scale: float, causal: bool,
+               stream=None) -> None:
+    """Forward with e4m3 inputs (uint8 or float8_e4m3fn tensors) and per-tensor descales."""
+    B, H, N, d = _shape(q8)
+    for t in (q8, k8, v8):
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or tuple(t.shape) != (B, H, N, d) \
+                or not t.is_contiguous() or t.device.type != "cuda":
+            raise ValueError("e4m3 inputs must be contiguous CUDA uint8/float8_e4m3fn [B,H,N,d]")
+    _check_tensors((B, H, N, d), torch.bfloat16, o)
+    _check_tensors((B, H, N), torch.float32, lse)
+    check(lib.fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_descale), float(k_descale), float(v_descale),
+                         _ptr(o), _ptr(lse), B, H, N, d, float(scale), int(bool(causal)), _stream_ptr(stream)))
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    n = int(lib.fa_bwd_workspace_size(B, H, N, d))
+    if n == ctypes.c_size_t(-1).value:
+        raise FAError(1, "invalid shape for fa_bwd_workspace_size")
+    return n
+
+
+def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, workspace, stream=None) -> None:
+    """dQ, dK, dV <- backward of attention; workspace is a CUDA uint8 tensor."""
+    B, H, N, d = _shape(q)
+    _check_tensors((B, H, N, d), torch.bfloat16, q, k, v, o, do, dq, dk, dv)
+    _check_tensors((B, H, N), torch.float32, lse)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                     B, H, N, d, float(scale), int(bool(causal)), _ptr(workspace), wbytes, _stream_ptr(stream)))
+
+
+def fa_device_status(stream=None):
+    """(status, where) of the device status word; synchronises the stream and clears it."""
+    where = ctypes.c_uint32(0)
+    st = lib.fa_device_status(_stream_ptr(stream), ctypes.byref(where))
+    return st, int(where.value)
+
+
+def fa_watchdog_selftest(limit_us: int, stream=None) -> None:
+    check(lib.fa_watchdog_selftest(int(limit_us), _stream_ptr(stream)))
+
+
+def _default_scale(d: int) -> float:
+    return d ** -0.5
+
+
+def attention_forward(q, k, v, scale: float | None = None, causal: bool = False, stream=None):
+    """Allocates O (bf16) and LSE (fp32) with torch and runs fa_fwd."""
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, o, lse, _default_scale(d) if scale is None else scale, causal, stream)
+    return o, lse
+
+
+def attention_forward_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale: float | None = None,
+                          causal: bool = False, stream=None):
+    B, H, N, d = _shape(q8)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    fa_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, o, lse,
+               _default_scale(d) if scale is None else scale, causal, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, do, lse, scale: float | None = None, causal: bool = False, workspace=None,
+                       stream=None):
+    """Allocates dQ, dK, dV (and the workspace unless given) with torch and runs fa_bwd."""
+    B, H, N, d = _shape(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(max(1, fa_bwd_workspace_size(B, H, N, d)), dtype=torch.uint8, device=q.device)
+    fa_bwd(q, k, v, o, do, lse, dq, dk, dv, _default_scale(d) if scale is None else scale, causal, workspace,
+           stream)
+    return dq, dk, dv

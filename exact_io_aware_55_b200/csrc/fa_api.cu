@@ -1,0 +1,268 @@
+// C ABI of the library (declared in include/fa.h): argument checks, TMA
+// tensor-map construction and kernel dispatch.  No allocation, no
+// synchronisation (except fa_device_status, which documents it).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace {
+
+// Status words (code, where) written by bounded waits that run out.
+__device__ uint32_t g_status_words[2];
+
+__global__ void watchdog_selftest_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    fa::mbar_init(&bar, 1);
+    abort_flag = 0u;
+    fa::fence_mbar_init();
+  }
+  __syncthreads();
+  const fa::WaitCtx wc{&abort_flag, status, limit_ns};
+  // Nobody arrives on `bar`: the wait must end through its time limit.
+  (void)fa::mbar_wait_warp(&bar, 0, wc, fa::WAIT_SELFTEST);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_arch_ok[kMaxDevices];  // 0 unknown, 1 sm_100, 2 other
+uint32_t* g_status_ptr[kMaxDevices];
+
+// Checks that the current device is an sm_100 part and returns its status
+// word address.
+fa_status current_device(uint32_t** status) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_ARCH;
+  int known = g_arch_ok[dev].load(std::memory_order_acquire);
+  if (known == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FA_ERR_ARCH;
+    void* sp = nullptr;
+    if (major == 10 && minor == 0 && cudaGetSymbolAddress(&sp, g_status_words) == cudaSuccess) {
+      g_status_ptr[dev] = static_cast<uint32_t*>(sp);
+      known = 1;
+    } else {
+      known = 2;
+    }
+    g_arch_ok[dev].store(known, std::memory_order_release);
+  }
+  if (known != 1) return FA_ERR_ARCH;
+  *status = g_status_ptr[dev];
+  return FA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// 3-D tensor map over a contiguous [BH, N, d] tensor: dims {d, N, BH},
+// box {128 bytes of d, 128 rows, 1 head}, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* map, const void* base, bool e4m3, int d, int N, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int eb = e4m3 ? 1 : 2;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * eb, cuuint64_t(N) * d * eb};
+  cuuint32_t box[3] = {cuuint32_t(128 / eb), 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Shape checks shared by every entry point.  Sets *empty when there is
+// nothing to compute.
+fa_status check_shape(int B, int H, int N, int d, float scale, int causal, bool* empty) {
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.0f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > 65535) return FA_ERR_UNSUPPORTED;  // grid.x limit of the launch shape
+  // Element offsets are computed in 64-bit; per-head rows in 32-bit.
+  if (static_cast<long long>(N) * d > (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  *empty = (BH == 0 || N == 0);
+  return FA_OK;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+size_t padded_rows(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
+
+struct WsLayout {
+  size_t dvec_off, lse2_off, dq_off, total;
+};
+WsLayout ws_layout(long long BH, int N, int d) {
+  WsLayout w{};
+  const size_t rows = static_cast<size_t>(BH) * padded_rows(N);
+  w.dvec_off = 0;
+  w.lse2_off = (rows * 4 + 255) / 256 * 256;
+  w.dq_off = w.lse2_off + (rows * 4 + 255) / 256 * 256;
+  w.total = w.dq_off + static_cast<size_t>(BH) * N * d * 4;
+  return w;
+}
+
+fa_status launch_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH; }
+
+fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                     float scale, int causal, void* stream, bool e4m3, float qd, float kd, float vd) {
+  bool empty = false;
+  fa_status st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK) return st;
+  if (e4m3 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (e4m3 && !(std::isfinite(qd) && std::isfinite(kd) && std::isfinite(vd) && qd > 0 && kd > 0 && vd > 0))
+    return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGNMENT;
+  uint32_t* status = nullptr;
+  if ((st = current_device(&status)) != FA_OK) return st;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, e4m3, d, N, BH) || !make_map(&tk, k, e4m3, d, N, BH) || !make_map(&tv, v, e4m3, d, N, BH))
+    return FA_ERR_LAUNCH;
+  fa::FwdArgs a{};
+  a.status = status;
+  a.o = o;
+  a.lse = lse;
+  a.N = N;
+  a.BH = BH;
+  a.c_log2 = scale * kLog2e * (e4m3 ? qd * kd : 1.0f);
+  a.o_scale = e4m3 ? vd : 1.0f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return launch_status(e4m3 ? fa::launch_fwd_e4m3(tq, tk, tv, a, d, causal != 0, s)
+                            : fa::launch_fwd_bf16(tq, tk, tv, a, d, causal != 0, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, void* stream) {
+  return fwd_common(q, k, v, o, lse, B, H, N, d, scale, causal, stream, false, 1.f, 1.f, 1.f);
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_descale, float k_descale,
+                     float v_descale, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
+                     void* stream) {
+  return fwd_common(q8, k8, v8, o, lse, B, H, N, d, scale, causal, stream, true, q_descale, k_descale, v_descale);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  bool empty = false;
+  if (check_shape(B, H, N, d, 1.0f, 0, &empty) != FA_OK) return static_cast<size_t>(-1);
+  if (empty) return 0;
+  return ws_layout(static_cast<long long>(B) * H, N, d).total;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  bool empty = false;
+  fa_status st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK) return st;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  const int BH = B * H;
+  const WsLayout wl = ws_layout(BH, N, d);
+  if (!workspace || workspace_bytes < wl.total) return FA_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(workspace, 16) || !aligned(lse, 4))
+    return FA_ERR_ALIGNMENT;
+  uint32_t* status = nullptr;
+  if ((st = current_device(&status)) != FA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, false, d, N, BH) || !make_map(&tk, k, false, d, N, BH) ||
+      !make_map(&tv, v, false, d, N, BH) || !make_map(&tdo, dO, false, d, N, BH))
+    return FA_ERR_LAUNCH;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  fa::BwdArgs a{};
+  a.status = status;
+  a.o = o;
+  a.dO = dO;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dvec = reinterpret_cast<float*>(ws + wl.dvec_off);
+  a.lse2 = reinterpret_cast<float*>(ws + wl.lse2_off);
+  a.dq_acc = reinterpret_cast<float*>(ws + wl.dq_off);
+  a.N = N;
+  a.Np = static_cast<int>(padded_rows(N));
+  a.BH = BH;
+  a.c_log2 = scale * kLog2e;
+  a.scale = scale;
+  return launch_status(fa::launch_bwd(tq, tk, tv, tdo, a, d, causal != 0, static_cast<cudaStream_t>(stream)));
+}
+
+const char* fa_strerror(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size, bad scale or causal flag)";
+    case FA_ERR_UNSUPPORTED: return "unsupported shape (head dimension must be 64 or 128; e4m3 needs 128)";
+    case FA_ERR_ALIGNMENT: return "misaligned pointer (tensors need 16-byte, lse 4-byte alignment)";
+    case FA_ERR_ARCH: return "current CUDA device is not an sm_100 (B200-class) GPU";
+    case FA_ERR_LAUNCH: return "CUDA launch or tensor-map setup failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    case FA_ERR_WORKSPACE: return "backward workspace missing or smaller than fa_bwd_workspace_size()";
+  }
+  return "unknown fa_status";
+}
+
+fa_status fa_device_status(void* stream, uint32_t* where) {
+  uint32_t* status = nullptr;
+  fa_status st = current_device(&status);
+  if (st != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t host[2] = {0u, 0u};
+  if (cudaMemcpyAsync(host, status, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (cudaMemsetAsync(status, 0, sizeof(host), s) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (where) *where = host[1];
+  return host[0] == 0u ? FA_OK : FA_ERR_DEVICE_TIMEOUT;
+}
+
+fa_status fa_watchdog_selftest(uint32_t limit_us, void* stream) {
+  if (limit_us == 0u || limit_us > 1000000u) return FA_ERR_INVALID_ARG;
+  uint32_t* status = nullptr;
+  fa_status st = current_device(&status);
+  if (st != FA_OK) return st;
+  watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status,
+                                                                             uint64_t(limit_us) * 1000ull);
+  return launch_status(cudaGetLastError());
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

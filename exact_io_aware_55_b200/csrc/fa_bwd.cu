@@ -1,0 +1,502 @@
+// Backward kernels of exact IO-aware attention for sm_100a.
+//
+// Method (explainers.rudrite.com "flash-attention-anatomy", Q&A "How does
+// FlashAttention save memory in the backward pass?"; kipu-akw.pages.dev "The
+// Real Complexity", recomputation on the backward pass): P is never stored; each
+// tile of S and P is recomputed from Q, K and the saved per-row LSE, and the
+// gradients follow from the chain rule through O = P V, P = softmax(S),
+// S = scale Q K^T:
+//   D = rowsum(dO o O), dV = P^T dO, dP = dO V^T, dS = P o (dP - D),
+//   dQ = scale dS K, dK = scale dS^T Q.
+//
+// Three launches on the caller's stream:
+//   bwd_pre      D and LSE*log2(e) per row (padded to 128-row tiles, +inf LSE on
+//                padding rows so their P is exactly 0) and zeroing of the fp32
+//                dQ accumulator.
+//   bwd_kernel   one CTA per (key tile j, batch-head); K_j, V_j stay in shared
+//                memory, dK_j and dV_j accumulate in TMEM, and the CTA walks the
+//                query tiles i (from the diagonal when causal):
+//                  S^T = K_j Q_i^T      -> TMEM R1       (tcgen05, smem x smem)
+//                  dP^T = V_j dO_i^T    -> TMEM R2
+//                  P^T = exp2(S^T c - LSE2_i)  written back over R1 as bf16
+//                  dV_j += P^T dO_i     (A = P^T from TMEM)
+//                  dS^T = scale P^T o (dP^T - D_i) -> shared memory (bf16, swizzled)
+//                  dK_j += dS^T Q_i     (A = dS^T, K-major)
+//                  dQ_i  = dS K_j       -> TMEM R2 (A = the same dS^T bytes read
+//                                          MN-major), then fp32 red.add into the
+//                                          workspace accumulator
+//   bwd_dq_final dQ accumulator -> bf16.
+// Warp roles in bwd_kernel: 0 TMA producer, 1 MMA issuer (+TMEM owner),
+// 4-7 the P / dS warpgroup (thread = key row = TMEM lane), 8-11 the dQ
+// warpgroup (thread = query row).  Epilogue: warps 4-7 store dV, 8-11 dK.
+// TMEM columns: dV [0,d) dK [d,2d) R1 [2d,2d+128) R2 [2d+128,2d+256).
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fa {
+
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------- preprocess
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a, int row_blocks, long long dq_vec4) {
+  constexpr int TPR = D / 8;              // threads per row, 8 elements (16 B) each
+  constexpr int RPB = 256 / TPR;          // rows per block
+  if (int(blockIdx.x) < row_blocks) {
+    const int row = blockIdx.x * RPB + threadIdx.x / TPR;   // row in [0, BH*Np)
+    const int sub = threadIdx.x % TPR;
+    const int bh = row / a.Np;
+    const int i = row - bh * a.Np;
+    const bool in_range = bh < a.BH;     // always true: BH*Np is a multiple of RPB
+    float part = 0.0f;
+    if (in_range && i < a.N) {
+      const size_t off = (size_t(bh) * a.N + i) * D + sub * 8;
+      const uint4 ov = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.o) + off);
+      const uint4 gv = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.dO) + off);
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 of = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[t]));
+        const float2 gf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[t]));
+        part = fmaf(of.x, gf.x, part);
+        part = fmaf(of.y, gf.y, part);
+      }
+    }
+#pragma unroll
+    for (int m = TPR / 2; m > 0; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+    if (sub == 0 && in_range) {
+      const size_t r = size_t(bh) * a.Np + i;
+      a.dvec[r] = (i < a.N) ? part : 0.0f;
+      a.lse2[r] = (i < a.N) ? a.lse[size_t(bh) * a.N + i] * kLog2e : INFINITY;
+    }
+  } else {
+    const long long stride = (long long)(gridDim.x - row_blocks) * blockDim.x;
+    float4* acc = reinterpret_cast<float4*>(a.dq_acc);
+    for (long long t = (long long)(blockIdx.x - row_blocks) * blockDim.x + threadIdx.x; t < dq_vec4; t += stride)
+      acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// ------------------------------------------------------------ dQ finalize
+__global__ void __launch_bounds__(256) bwd_dq_final_kernel(const float* __restrict__ acc, __nv_bfloat16* dq,
+                                                           long long n8) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n8; t += stride) {
+    const float4 x = reinterpret_cast<const float4*>(acc)[2 * t];
+    const float4 y = reinterpret_cast<const float4*>(acc)[2 * t + 1];
+    uint4 o;
+    o.x = pack_bf16x2(x.x, x.y);
+    o.y = pack_bf16x2(x.z, x.w);
+    o.z = pack_bf16x2(y.x, y.y);
+    o.w = pack_bf16x2(y.z, y.w);
+    reinterpret_cast<uint4*>(dq)[t] = o;
+  }
+}
+
+// ---------------------------------------------------------------- main
+template <int D>
+struct BwdShape {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kChunks = kRowBytes / 128;
+  static constexpr int kTileBytes = 128 * kRowBytes;     // one 128-row bf16 tile
+  static constexpr int kDsBytes = 128 * 128 * 2;         // dS^T: 128 keys x 128 queries, bf16 (any d)
+  static constexpr int kNST = 2;                         // Q/dO ring depth
+  static constexpr int kKSteps = kRowBytes / 32;         // K-steps over d (16 elements)
+  static constexpr uint32_t kIdSS = idesc_bf16(128, 128, false, false);   // S^T, dP^T
+  static constexpr uint32_t kIdKmaj = idesc_bf16(128, D, false, true);    // dV, dK: B MN-major
+  static constexpr uint32_t kIdDQ = idesc_bf16(128, D, true, true);       // dQ: A and B MN-major
+  static constexpr uint32_t kColDV = 0, kColDK = D, kColR1 = 2 * D, kColR2 = 2 * D + 128;
+};
+
+template <int NST>
+struct BwdBarriers {
+  uint64_t kv_full;
+  uint64_t qdo_full[NST];
+  uint64_t qdo_empty[NST];
+  uint64_t s_ready, dp_ready, p_ready, ds_ready, ds_free, dq_ready, dq_free, final_;
+  uint32_t tmem_base;
+  uint32_t abort;
+};
+
+template <int D>
+constexpr size_t bwd_smem_bytes() {
+  using S = BwdShape<D>;
+  return size_t(2 + 2 * S::kNST) * S::kTileBytes + S::kDsBytes + S::kNST * 1024 + sizeof(BwdBarriers<S::kNST>);
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+               const BwdArgs args) {
+  using S = BwdShape<D>;
+  constexpr int NST = S::kNST;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  auto* bars =
+      reinterpret_cast<BwdBarriers<NST>*>(smem + (2 + 2 * NST) * S::kTileBytes + S::kDsBytes + NST * 1024);
+  // The layout relies on a 1024-byte aligned dynamic shared-memory base (the
+  // 128-byte swizzle atoms); refuse to run otherwise.
+  if ((smem_u32(smem) & 1023u) != 0u) {
+    if (threadIdx.x == 0) {
+      atomicCAS(&args.status[0], DEVSTATUS_OK, DEVSTATUS_WAIT_TIMEOUT);
+      atomicExch(&args.status[1], WAIT_BWD_FINAL);
+    }
+    return;
+  }
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + S::kTileBytes;
+  uint8_t* sQ = sV + S::kTileBytes;                 // NST tiles
+  uint8_t* sdO = sQ + NST * S::kTileBytes;          // NST tiles
+  uint8_t* sdS = sdO + NST * S::kTileBytes;         // dS^T: rows = keys, 128 queries each
+  float* sStat = reinterpret_cast<float*>(sdS + S::kDsBytes);     // per stage: lse2[128], D[128]
+  const WaitCtx wc{&bars->abort, args.status, FA_WAIT_LIMIT_NS};
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int j = blockIdx.y;                          // key tile
+  const int N = args.N;
+  const int n_q = (N + kTile - 1) / kTile;
+  const int i_begin = CAUSAL ? j : 0;
+  const int n_iter = n_q - i_begin;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&bars->qdo_full[s], 1);
+      mbar_init(&bars->qdo_empty[s], 1 + 4);
+    }
+    mbar_init(&bars->s_ready, 1);
+    mbar_init(&bars->dp_ready, 1);
+    mbar_init(&bars->p_ready, 4);
+    mbar_init(&bars->ds_ready, 4);
+    mbar_init(&bars->ds_free, 1);
+    mbar_init(&bars->dq_ready, 1);
+    mbar_init(&bars->dq_free, 4);
+    mbar_init(&bars->final_, 1);
+    bars->abort = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      const uint64_t pol_q = policy_evict_last();    // Q/dO tiles are re-read by every key tile
+      const uint64_t pol_kv = policy_evict_first();  // K/V tiles are read once
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * S::kTileBytes);
+      for (int c = 0; c < S::kChunks; ++c) {
+        tma_load_3d_hint(sK + c * 16384, &tmK, &bars->kv_full, c * 64, j * kTile, bh, pol_kv);
+        tma_load_3d_hint(sV + c * 16384, &tmV, &bars->kv_full, c * 64, j * kTile, bh, pol_kv);
+      }
+      for (int it = 0; it < n_iter; ++it) {
+        const int s = it % NST;
+        const int i = i_begin + it;
+        if (it >= NST) {
+          if (!mbar_wait(&bars->qdo_empty[s], ((it / NST) + 1) & 1, wc, WAIT_BWD_QDO_EMPTY)) break;
+        }
+        mbar_arrive_expect_tx(&bars->qdo_full[s], 2 * S::kTileBytes + 1024);
+        for (int c = 0; c < S::kChunks; ++c) {
+          tma_load_3d_hint(sQ + s * S::kTileBytes + c * 16384, &tmQ, &bars->qdo_full[s], c * 64, i * kTile, bh,
+                           pol_q);
+          tma_load_3d_hint(sdO + s * S::kTileBytes + c * 16384, &tmdO, &bars->qdo_full[s], c * 64, i * kTile,
+                           bh, pol_q);
+        }
+        const size_t srow = size_t(bh) * args.Np + size_t(i) * kTile;
+        bulk_load(sStat + s * 256, args.lse2 + srow, 512, &bars->qdo_full[s]);
+        bulk_load(sStat + s * 256 + 128, args.dvec + srow, 512, &bars->qdo_full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sdOa = smem_u32(sdO),
+                     sdSa = smem_u32(sdS);
+      const uint32_t tR1 = tmem + S::kColR1, tR2 = tmem + S::kColR2;
+      // X^T tile = A_tile B_tile^T over d, both K-major (S^T = K Q^T, dP^T = V dO^T).
+      auto issue_xt = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+        for (int ks = 0; ks < S::kKSteps; ++ks) {
+          const uint32_t off = uint32_t((ks >> 2) * 16384 + (ks & 3) * 32);
+          mma_f16_ss(d_tmem, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024), S::kIdSS,
+                     ks > 0);
+        }
+      };
+      bool ok = mbar_wait(&bars->kv_full, 0, wc, WAIT_BWD_KV) && mbar_wait(&bars->qdo_full[0], 0, wc, WAIT_BWD_QDO);
+      if (ok) {
+        tc_fence_after();
+        issue_xt(tR1, sKa, sQa);                       // S^T_0
+        tc_commit(&bars->s_ready);
+        for (int it = 0; it < n_iter; ++it) {
+          const int s = it % NST;
+          const uint32_t qa = sQa + s * S::kTileBytes, doa = sdOa + s * S::kTileBytes;
+          if (it > 0) {
+            if (!mbar_wait(&bars->dq_free, (it - 1) & 1, wc, WAIT_BWD_DQ_FREE)) { ok = false; break; }
+            tc_fence_after();
+          }
+          issue_xt(tR2, sVa, doa);                     // dP^T_it
+          tc_commit(&bars->dp_ready);
+          if (!mbar_wait(&bars->p_ready, it & 1, wc, WAIT_BWD_P)) { ok = false; break; }
+          tc_fence_after();
+          // dV += P^T dO: A = P^T (TMEM R1, bf16), B = dO MN-major; 16 queries per step.
+#pragma unroll
+          for (int kt = 0; kt < 8; ++kt)
+            mma_f16_ts(tmem + S::kColDV, tR1 + kt * 8, sdesc_sw128(doa + kt * 2048, 16384, 1024), S::kIdKmaj,
+                       (it > 0 || kt > 0) ? 1u : 0u);
+          if (it + 1 < n_iter) {                        // S^T of the next query tile
+            const int sn = (it + 1) % NST;
+            if (!mbar_wait(&bars->qdo_full[sn], ((it + 1) / NST) & 1, wc, WAIT_BWD_QDO)) { ok = false; break; }
+            tc_fence_after();
+            issue_xt(tR1, sKa, sQa + sn * S::kTileBytes);
+            tc_commit(&bars->s_ready);
+          }
+          if (!mbar_wait(&bars->ds_ready, it & 1, wc, WAIT_BWD_DS)) { ok = false; break; }
+          tc_fence_after();
+          // dK += dS^T Q: A = dS^T K-major (rows = keys, 128 queries), B = Q MN-major.
+#pragma unroll
+          for (int kt = 0; kt < 8; ++kt) {
+            const uint32_t off = uint32_t((kt >> 2) * 16384 + (kt & 3) * 32);
+            mma_f16_ss(tmem + S::kColDK, sdesc_sw128(sdSa + off, 16, 1024),
+                       sdesc_sw128(qa + kt * 2048, 16384, 1024), S::kIdKmaj, (it > 0 || kt > 0) ? 1u : 0u);
+          }
+          // dQ = dS K: A = the dS^T bytes read MN-major (M = queries), B = K MN-major; 16 keys per step.
+#pragma unroll
+          for (int kt = 0; kt < 8; ++kt)
+            mma_f16_ss(tR2, sdesc_sw128(sdSa + kt * 2048, 16384, 1024), sdesc_sw128(sKa + kt * 2048, 16384, 1024),
+                       S::kIdDQ, kt > 0 ? 1u : 0u);
+          tc_commit(&bars->dq_ready);
+          tc_commit(&bars->ds_free);
+          tc_commit(&bars->qdo_empty[s]);
+        }
+        tc_commit(&bars->final_);
+        if (ok) (void)mbar_wait(&bars->final_, 0, wc, WAIT_BWD_FINAL);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------- P / dS group
+    const int wq = warp & 3;
+    const int c = wq * 32 + lane;                   // key row within the tile
+    const int kv = j * kTile + c;
+    const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
+    const uint32_t tR1 = lane_base + S::kColR1, tR2 = lane_base + S::kColR2;
+    const float cl = args.c_log2;
+    const float scale = args.scale;
+    const bool kv_valid = kv < N;
+    bool ok = true;
+    for (int it = 0; it < n_iter && ok; ++it) {
+      const int s = it % NST;
+      const int i = i_begin + it;
+      const float* sl = sStat + s * 256;            // lse2 of the 128 queries
+      const float* sd = sl + 128;                   // D of the 128 queries
+      // LSE2 / D of this stage arrived by bulk copy on qdo_full; S^T by MMA commit.
+      if (!mbar_wait_warp(&bars->qdo_full[s], (it / NST) & 1, wc, WAIT_BWD_QDO)) { ok = false; break; }
+      if (!mbar_wait_warp(&bars->s_ready, it & 1, wc, WAIT_BWD_S)) { ok = false; break; }
+      tc_fence_after();
+      // P^T row: exp2(S^T * scale * log2e - LSE2_q); masked entries are 0.
+      const bool diag = CAUSAL && (i == j);
+      uint32_t pk[64];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t r[32];
+        tmem_ld_x32(tR1 + q4 * 32, r);
+        uint32_t w[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int q0 = q4 * 32 + 2 * t;
+          float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * t]), cl, -sl[q0]));
+          float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * t + 1]), cl, -sl[q0 + 1]));
+          if (diag) {
+            if (c > q0) p0 = 0.0f;
+            if (c > q0 + 1) p1 = 0.0f;
+          }
+          if (!kv_valid) p0 = p1 = 0.0f;
+          w[t] = pack_bf16x2(p0, p1);
+          pk[q4 * 16 + t] = w[t];
+        }
+        tmem_st_x16(tR1 + q4 * 16, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_ready);
+      // dS^T row = scale * P^T o (dP^T - D_q) -> shared memory, 128-byte swizzled K-major rows.
+      if (!mbar_wait_warp(&bars->dp_ready, it & 1, wc, WAIT_BWD_DP)) { ok = false; break; }
+      if (it > 0 && !mbar_wait_warp(&bars->ds_free, (it - 1) & 1, wc, WAIT_BWD_DS_FREE)) { ok = false; break; }
+      tc_fence_after();
+      uint8_t* row_base = sdS + (c >> 3) * 1024 + (c & 7) * 128;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t r[32];
+        tmem_ld_x32(tR2 + q4 * 32, r);
+        uint32_t w[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int q0 = q4 * 32 + 2 * t;
+          const uint32_t pw = pk[q4 * 16 + t];
+          const float ds0 = scale * bf16lo(pw) * (__uint_as_float(r[2 * t]) - sd[q0]);
+          const float ds1 = scale * bf16hi(pw) * (__uint_as_float(r[2 * t + 1]) - sd[q0 + 1]);
+          w[t] = pack_bf16x2(ds0, ds1);
+        }
+        // 32 queries = 64 bytes = four 16-byte units of chunk (q4 >> 1).
+        uint8_t* chunk = row_base + (q4 >> 1) * 16384;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = (q4 & 1) * 4 + u;
+          *reinterpret_cast<uint4*>(chunk + ((unit ^ (c & 7)) << 4)) =
+              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->ds_ready);
+        mbar_arrive(&bars->qdo_empty[s]);           // done with this stage's LSE2 / D
+      }
+    }
+    // dV epilogue
+    if (ok && mbar_wait_warp(&bars->final_, 0, wc, WAIT_BWD_FINAL)) {
+      tc_fence_after();
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.dv) + (size_t(bh) * N + kv) * D;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t r[32];
+        tmem_ld_x32(lane_base + S::kColDV + q * 32, r);
+        if (kv_valid) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]), __uint_as_float(r[8 * u + 1]));
+            v.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]), __uint_as_float(r[8 * u + 3]));
+            v.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]), __uint_as_float(r[8 * u + 5]));
+            v.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]), __uint_as_float(r[8 * u + 7]));
+            reinterpret_cast<uint4*>(dst + q * 32)[u] = v;
+          }
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ---------------------------------------------------------- dQ group
+    const int wq = warp & 3;
+    const int r0 = wq * 32 + lane;                  // query row within the tile (dQ) / key row (dK)
+    const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
+    bool ok = true;
+    for (int it = 0; it < n_iter; ++it) {
+      const int i = i_begin + it;
+      if (!mbar_wait_warp(&bars->dq_ready, it & 1, wc, WAIT_BWD_DQ)) { ok = false; break; }
+      tc_fence_after();
+      float dq[D];
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t r[32];
+        tmem_ld_x32(lane_base + S::kColR2 + q * 32, r);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) dq[q * 32 + t] = __uint_as_float(r[t]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->dq_free);
+      const int qrow = i * kTile + r0;
+      if (qrow < N) {
+        float* dst = args.dq_acc + (size_t(bh) * N + qrow) * D;
+#pragma unroll
+        for (int t = 0; t < D / 4; ++t) red_add_v4(dst + 4 * t, dq[4 * t], dq[4 * t + 1], dq[4 * t + 2], dq[4 * t + 3]);
+      }
+    }
+    // dK epilogue
+    if (ok && mbar_wait_warp(&bars->final_, 0, wc, WAIT_BWD_FINAL)) {
+      tc_fence_after();
+      const int kv = j * kTile + r0;
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.dk) + (size_t(bh) * N + kv) * D;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t r[32];
+        tmem_ld_x32(lane_base + S::kColDK + q * 32, r);
+        if (kv < N) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]), __uint_as_float(r[8 * u + 1]));
+            v.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]), __uint_as_float(r[8 * u + 3]));
+            v.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]), __uint_as_float(r[8 * u + 5]));
+            v.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]), __uint_as_float(r[8 * u + 7]));
+            reinterpret_cast<uint4*>(dst + q * 32)[u] = v;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
+  // 1) preprocess + zero the dQ accumulator
+  constexpr int RPB = 256 / (D / 8);
+  const long long rows = (long long)a.BH * a.Np;
+  const int row_blocks = int((rows + RPB - 1) / RPB);
+  const long long dq_vec4 = (long long)a.BH * a.N * D / 4;
+  const int zero_blocks = int(std::min<long long>((dq_vec4 + 255) / 256, 148LL * 8));
+  bwd_pre_kernel<D><<<row_blocks + zero_blocks, 256, 0, stream>>>(a, row_blocks, dq_vec4);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // 2) main kernel
+  constexpr size_t smem = bwd_smem_bytes<D>();
+  auto kern = bwd_kernel<D, CAUSAL>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.BH, (a.N + kTile - 1) / kTile);
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // 3) dQ -> bf16
+  const long long n8 = (long long)a.BH * a.N * D / 8;
+  const int fin_blocks = int(std::min<long long>((n8 + 255) / 256, 148LL * 8));
+  bwd_dq_final_kernel<<<fin_blocks, 256, 0, stream>>>(a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq), n8);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                       const BwdArgs& a, int d, bool causal, cudaStream_t stream) {
+  if (d == 64) return causal ? launch_bwd_t<64, true>(tq, tk, tv, tdo, a, stream)
+                             : launch_bwd_t<64, false>(tq, tk, tv, tdo, a, stream);
+  return causal ? launch_bwd_t<128, true>(tq, tk, tv, tdo, a, stream)
+                : launch_bwd_t<128, false>(tq, tk, tv, tdo, a, stream);
+}
+
+}  // namespace fa

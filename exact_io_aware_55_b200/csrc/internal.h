@@ -1,0 +1,71 @@
+// Internal launch interface between the C ABI (fa_api.cu) and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace fa {
+
+// Codes recorded in the device status "where" word by a bounded wait that ran out.
+enum WaitSite : uint32_t {
+  WAIT_FWD_Q = 1,
+  WAIT_FWD_K = 2,
+  WAIT_FWD_V = 3,
+  WAIT_FWD_KV_EMPTY = 4,
+  WAIT_FWD_S = 5,
+  WAIT_FWD_P = 6,
+  WAIT_FWD_O = 7,
+  WAIT_BWD_KV = 16,
+  WAIT_BWD_QDO = 17,
+  WAIT_BWD_QDO_EMPTY = 18,
+  WAIT_BWD_S = 19,
+  WAIT_BWD_DP = 20,
+  WAIT_BWD_P = 21,
+  WAIT_BWD_DS = 22,
+  WAIT_BWD_DS_FREE = 23,
+  WAIT_BWD_DQ = 24,
+  WAIT_BWD_DQ_FREE = 25,
+  WAIT_BWD_FINAL = 26,
+  WAIT_SELFTEST = 99,
+};
+
+struct FwdArgs {
+  uint32_t* status;   // device status words (code, where)
+  void* o;        // bf16 [BH, N, d]
+  float* lse;     // fp32 [BH, N]
+  int N;
+  int BH;
+  float c_log2;   // scale * log2(e), times the q/k descales for e4m3 inputs
+  float o_scale;  // factor applied with 1/l to O (1, or the v descale for e4m3)
+};
+
+struct BwdArgs {
+  uint32_t* status;   // device status words (code, where)
+  const void* o;      // bf16 [BH, N, d]
+  const void* dO;     // bf16 [BH, N, d]
+  const float* lse;   // fp32 [BH, N]
+  void* dq;           // bf16 [BH, N, d]
+  void* dk;           // bf16 [BH, N, d]
+  void* dv;           // bf16 [BH, N, d]
+  float* dvec;        // workspace: D, fp32 [BH, Np]
+  float* lse2;        // workspace: LSE * log2(e), fp32 [BH, Np] (+inf on padded rows)
+  float* dq_acc;      // workspace: fp32 [BH, N, d]
+  int N;
+  int Np;             // N rounded up to a multiple of 128
+  int BH;
+  float c_log2;       // scale * log2(e)
+  float scale;
+};
+
+// Tensor maps: 3-D views {d, N, BH} of a [BH, N, d] tensor, box {128 bytes, 128 rows, 1},
+// 128-byte swizzle, zero fill out of bounds.
+cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdArgs& a, int d, bool causal, cudaStream_t stream);
+cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdArgs& a, int d, bool causal, cudaStream_t stream);
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const BwdArgs& a, int d, bool causal, cudaStream_t stream);
+cudaError_t launch_watchdog_selftest(uint64_t limit_ns, cudaStream_t stream);
+
+}  // namespace fa

@@ -1,0 +1,153 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact IO-aware attention library.
+ *
+ * What the library computes is exact attention, O = softmax(scale * Q K^T) V,
+ * tiled so that the N x N scores S and probabilities P live only in on-chip
+ * memory (TMEM / shared memory) and are never written to HBM; the forward saves
+ * one per-row statistic and the backward recomputes P tile by tile from it.
+ * Sources: explainers.rudrite.com "flash-attention-anatomy" (Q&As "Why is
+ * attention memory-bound, and how does FlashAttention fix it?", "What is online
+ * softmax and how does tiling keep it exact?", "How does FlashAttention save
+ * memory in the backward pass?", "What changed between FlashAttention 1, 2, and
+ * 3?"); chipfoundryservices.com glossary "flash attention" ("Tiling plus an
+ * online softmax removes the round trip"); kipu-akw.pages.dev "flash-attention /
+ * where-it-matters" (section "The Real Complexity").
+ *
+ * Conventions shared by every entry point:
+ *   - Layout: contiguous [B, H, N, d] row-major, d innermost, for every
+ *     [.., N, d] tensor; LSE and other per-row values are contiguous [B, H, N].
+ *   - Device pointers.  The caller owns every buffer (including the backward
+ *     workspace); the library allocates no device or pinned memory, keeps no
+ *     pointer after a call returns, and never synchronises the stream.
+ *   - Tensor pointers (q, k, v, o, dO, dq, dk, dv, workspace) must be 16-byte
+ *     aligned; lse must be 4-byte aligned.
+ *   - d (head dimension) must be 64 or 128.  N >= 1 is arbitrary: ragged tails
+ *     are masked.  B, H, N == 0 is a valid empty call that launches nothing.
+ *   - causal != 0 selects top-left aligned causal masking (key j is visible to
+ *     query i iff j <= i; Nq == Nk == N).  Fully masked tiles are skipped.
+ *   - scale is the softmax scale (the configurations use 1/sqrt(d)).
+ *   - stream is a cudaStream_t passed as an opaque pointer (NULL = legacy
+ *     default stream).
+ *   - Arguments are checked on the host before anything is launched; a bad
+ *     argument returns an error code and launches nothing.  A launch failure
+ *     returns FA_ERR_LAUNCH.  Asynchronous device faults surface at the
+ *     caller's next synchronisation.  Every device-side wait is bounded; one
+ *     that runs out records a status readable with fa_device_status().
+ *   - Thread safety: calls are re-entrant; the first call on a device also
+ *     configures the kernels' shared-memory limits for that device.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fa_status {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,     /* null pointer, bad size or dimension, bad scale */
+  FA_ERR_UNSUPPORTED = 2,     /* head dimension other than 64 / 128 */
+  FA_ERR_ALIGNMENT = 3,       /* pointer not 16-byte (4-byte for lse) aligned */
+  FA_ERR_ARCH = 4,            /* current device is not sm_100 (B200 class) */
+  FA_ERR_LAUNCH = 5,          /* CUDA runtime rejected a launch or attribute */
+  FA_ERR_DEVICE_TIMEOUT = 6,  /* a bounded device wait ran out (fa_device_status) */
+  FA_ERR_WORKSPACE = 7        /* backward workspace missing or too small */
+} fa_status;
+
+/*
+ * Forward pass, bf16.
+ * Computes O = softmax(scale * Q K^T) V per (batch, head) with a running row
+ * maximum m and denominator l carried across key tiles and the partial output
+ * rescaled by exp(m_old - m_new) when m grows ("What is online softmax and how
+ * does tiling keep it exact?"); writes only O and LSE = m + ln l, never S or P
+ * ("How does FlashAttention save memory in the backward pass?": the per-row
+ * softmax statistics are the only residual).
+ *   q, k, v : in,  bf16 [B,H,N,d]
+ *   o       : out, bf16 [B,H,N,d]
+ *   lse     : out, fp32 [B,H,N], natural-log log-sum-exp of each score row
+ */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for this shape (0 when empty).
+ * The workspace holds D = rowsum(dO o O) and the log2-domain LSE, both fp32
+ * per row padded to a multiple of 128 rows, and the fp32 dQ accumulator.
+ * Returns (size_t)-1 when the arguments are invalid.
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass, bf16, for a loss L with dL/dO = dO.
+ * Recomputes S and P = exp(S - LSE) tile by tile from Q, K and the saved LSE
+ * instead of reading a stored P ("How does FlashAttention save memory in the
+ * backward pass?"; "The Real Complexity", recomputation on the backward pass),
+ * then forms D = rowsum(dO o O), dV = P^T dO, dP = dO V^T, dS = P o (dP - D),
+ * dQ = scale dS K, dK = scale dS^T Q (chain rule through S = scale Q K^T).
+ * dQ is accumulated across key tiles with fp32 atomics, so its low bits may
+ * differ from run to run.
+ *   q, k, v, o, dO : in,  bf16 [B,H,N,d]  (o: the forward's output)
+ *   lse            : in,  fp32 [B,H,N]    (the forward's LSE)
+ *   dq, dk, dv     : out, bf16 [B,H,N,d]
+ *   workspace      : scratch device memory of >= workspace_bytes bytes, at
+ *                    least fa_bwd_workspace_size(B,H,N,d); contents on entry
+ *                    are ignored and on exit are unspecified.  Must not be
+ *                    used by another call that overlaps this one on the GPU.
+ */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Forward pass with float8 e4m3 inputs and per-tensor scales ("What changed
+ * between FlashAttention 1, 2, and 3?": low-precision FP8 forward).
+ * The real inputs are q8 * q_descale, k8 * k_descale, v8 * v_descale.  The
+ * score and value descales are folded into the exponent argument and the
+ * final normalisation; P is rounded to e4m3 for the P V product while the
+ * denominator l is summed in fp32.
+ *   q8, k8, v8 : in,  e4m3 (fn) bytes [B,H,N,d]
+ *   o          : out, bf16 [B,H,N,d]
+ *   lse        : out, fp32 [B,H,N]
+ * d must be 128 or 64; causal is supported.
+ */
+FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_descale, float k_descale,
+                     float v_descale, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
+                     void* stream);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+FA_API const char* fa_strerror(fa_status status);
+
+/*
+ * Reads and clears the library's device status word on the current device.
+ * Synchronises `stream` first.  Returns FA_OK, or FA_ERR_DEVICE_TIMEOUT if a
+ * bounded wait inside a kernel ran out since the last call (the kernel then
+ * abandoned its tile and returned; its outputs are undefined).  *where, if
+ * not NULL, receives a code naming the wait that gave up.
+ */
+FA_API fa_status fa_device_status(void* stream, uint32_t* where);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one block that waits on a
+ * barrier nobody arrives at, with the given limit in microseconds (1..10^6),
+ * so the wait runs out and the status word is set.  Used by the tests to
+ * check that a stuck wait ends with a status, not a hang.
+ */
+FA_API fa_status fa_watchdog_selftest(uint32_t limit_us, void* stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -72,14 +72,15 @@ def quantize_e4m3(x: np.ndarray):
 
 
 def attention_inputs(B: int, H: int, N: int, d: int, seed: int, q_mult: float = 1.0,
-                     with_grad: bool = True, storage: str = "bf16"):
+                     with_grad: bool = True, storage: str = "bf16", want_f64: bool = True):
     """Seeded Q, K, V (and dO) for one attention configuration.
 
     ``storage`` is ``"bf16"`` (Q, K, V, dO rounded to bf16) or ``"e4m3"`` (Q, K,
     V quantised with per-tensor scales; no dO).  The returned dict holds, per
     tensor name, the raw storage bits (``"<name>_bits"``) and the exact float64
     values the device will see (``"<name>"``).  For e4m3 it also holds
-    ``"<name>_descale"``.
+    ``"<name>_descale"``.  With ``want_f64=False`` the float64 copies are
+    skipped (large shapes); ``head_f64`` converts one head on demand.
     """
     shape = (B, H, N, d)
     out = {"shape": shape, "seed": seed, "q_mult": q_mult, "storage": storage}
@@ -91,15 +92,25 @@ def attention_inputs(B: int, H: int, N: int, d: int, seed: int, q_mult: float = 
         if storage == "bf16":
             bits = to_bf16_bits(x)
             out[name + "_bits"] = bits
-            out[name] = bf16_bits_to_f64(bits)
+            if want_f64:
+                out[name] = bf16_bits_to_f64(bits)
         elif storage == "e4m3":
             bits, descale, deq = quantize_e4m3(x)
             out[name + "_bits"] = bits
             out[name + "_descale"] = descale
-            out[name] = deq
+            if want_f64:
+                out[name] = deq
         else:
             raise ValueError(f"unknown storage {storage!r}")
     return out
+
+
+def head_f64(inp, name: str, b: int, h: int) -> np.ndarray:
+    """Exact float64 values of one head of tensor ``name``."""
+    bits = inp[name + "_bits"][b, h]
+    if inp["storage"] == "bf16":
+        return bf16_bits_to_f64(bits)
+    return e4m3_bits_to_f64(bits) * inp[name + "_descale"]
 
 
 def attention_inputs_f32_to_bf16(B, H, N, d, seed):

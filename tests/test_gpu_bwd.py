@@ -1,0 +1,128 @@
+"""GPU parity of the bf16 backward (fa_bwd) against the fp64 oracle.
+
+The device backward consumes the device forward's O and LSE, as a caller
+would; the oracle computes everything from the same rounded Q, K, V, dO.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+fa = pytest.importorskip("exact_io_aware_55_b200")
+
+
+def _device_inputs(inp):
+    return tuple(gu.dev_bf16(inp[n + "_bits"]) for n in ("q", "k", "v", "do"))
+
+
+def _run(inp, causal, scale=None, guarded=False):
+    B, H, N, d = inp["shape"]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    q, k, v, do = _device_inputs(inp)
+    o, lse = fa.attention_forward(q, k, v, scale=scale, causal=causal)
+    if guarded:
+        gs = [gu.Guarded((B, H, N, d), torch.bfloat16) for _ in range(3)]
+        wsz = fa.fa_bwd_workspace_size(B, H, N, d)
+        wg = gu.Guarded((max(wsz, 16),), torch.uint8)
+        fa.fa_bwd(q, k, v, o, do, lse, gs[0].view, gs[1].view, gs[2].view, scale, causal, wg.view)
+        torch.cuda.synchronize()
+        assert all(g.intact() for g in gs) and wg.intact(), "write outside the output/workspace buffers"
+        dq, dk, dv = (g.view for g in gs)
+    else:
+        dq, dk, dv = fa.attention_backward(q, k, v, o, do, lse, scale=scale, causal=causal)
+        torch.cuda.synchronize()
+    assert fa.fa_device_status() == (0, 0)
+    return tuple(gu.to_f64(t) for t in (dq, dk, dv)), scale
+
+
+def _assert_grads(got, ref, what=""):
+    for name, g, r in zip(("dQ", "dK", "dV"), got, ref):
+        assert np.all(np.isfinite(g)), f"non-finite {name} {what}"
+        e = gu.rel_fro(g, r)
+        assert e <= gu.GRAD_REL_FRO, f"{name} rel-Frobenius {e:.3e} > {gu.GRAD_REL_FRO} {what}"
+
+
+SMALL = [(1, 1, 128, 64), (1, 2, 1, 64), (1, 1, 17, 128), (2, 1, 127, 64), (1, 1, 129, 128),
+         (1, 2, 300, 64), (1, 1, 300, 128), (2, 2, 513, 128), (1, 3, 1000, 64), (1, 1, 640, 128)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SMALL)
+def test_bwd_small_parity(shape, causal):
+    B, H, N, d = shape
+    inp = synth.attention_inputs(B, H, N, d, seed=200 + N + d)
+    got, scale = _run(inp, causal, guarded=True)
+    ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["do"], scale, causal)
+    _assert_grads(got, ref, f"{shape} causal={causal}")
+
+
+def test_bwd_pr1_reference_case():
+    inp = synth.attention_inputs_f32_to_bf16(1, 1, 128, 64, seed=1234)
+    got, scale = _run(inp, False, scale=1.0 / 8.0)
+    ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["do"], scale, False)
+    _assert_grads(got, ref)
+
+
+@pytest.mark.parametrize("mult", [8.0])
+def test_bwd_large_score_range(mult):
+    inp = synth.attention_inputs(1, 2, 1024, 128, seed=78, q_mult=mult)
+    for causal in (False, True):
+        got, scale = _run(inp, causal)
+        ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["do"], scale, causal)
+        _assert_grads(got, ref, f"mult={mult} causal={causal}")
+
+
+def test_bwd_config_b4_h16_n2048_d64_full():
+    inp = synth.attention_inputs(4, 16, 2048, 64, seed=1236)
+    got, scale = _run(inp, False)
+    ref = oracle.attention_backward(inp["q"], inp["k"], inp["v"], inp["do"], scale, False)
+    _assert_grads(got, ref)
+
+
+def _sampled(B, H, N, d, causal, seed, q_mult=1.0, n_heads=2, n_rows=16):
+    inp = synth.attention_inputs(B, H, N, d, seed=seed, q_mult=q_mult, want_f64=False)
+    (dq, dk, dv), scale = _run(inp, causal)
+    # sum identities on every head: sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i
+    do_sum = np.stack([synth.head_f64(inp, "do", b, h).sum(axis=0) for b in range(B) for h in range(H)])
+    dk_sum = dk.sum(axis=2).reshape(B * H, d)
+    dv_sum = dv.sum(axis=2).reshape(B * H, d)
+    dk_norm = np.linalg.norm(dk.reshape(B * H, -1), axis=1)[:, None]
+    assert np.max(np.abs(dk_sum) / dk_norm) <= 1e-2
+    assert np.max(np.abs(dv_sum - do_sum) / np.linalg.norm(do_sum, axis=1)[:, None]) <= 1e-2
+    rng = np.random.default_rng(seed)
+    heads = {(0, 0), (B - 1, H - 1)}
+    while len(heads) < min(n_heads, B * H):
+        heads.add((int(rng.integers(B)), int(rng.integers(H))))
+    for (b, h) in sorted(heads):
+        rows = gu.sample_rows(N, n_rows, seed + 7 * b + h)
+        cols = gu.sample_rows(N, n_rows, seed + 11 * b + h + 1)
+        qh, kh, vh, doh = (synth.head_f64(inp, n, b, h) for n in ("q", "k", "v", "do"))
+        rq, rk, rv = oracle.head_backward_sampled(qh, kh, vh, doh, scale, causal, rows, cols)
+        _assert_grads((dq[b, h][rows], dk[b, h][cols], dv[b, h][cols]), (rq, rk, rv), f"head ({b},{h})")
+
+
+@pytest.mark.parametrize("q_mult", [1.0, 8.0])
+def test_bwd_config_b2_h16_n8192_d128_causal_sampled(q_mult):
+    _sampled(2, 16, 8192, 128, True, seed=1237, q_mult=q_mult)
+
+
+def test_bwd_config_b1_h32_n32768_d128_causal_sampled():
+    _sampled(1, 32, 32768, 128, True, seed=1238, n_heads=1, n_rows=12)
+
+
+def test_bwd_workspace_checks():
+    x = torch.zeros((1, 1, 64, 64), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, 1, 64), dtype=torch.float32, device="cuda")
+    outs = [torch.empty_like(x) for _ in range(3)]
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fa.FAError) as e:
+        fa.fa_bwd(x, x, x, x, x, lse, *outs, 0.125, False, small)
+    assert e.value.status == fa.STATUS_CODES["FA_ERR_WORKSPACE"]
+    assert fa.fa_bwd_workspace_size(1, 1, 0, 64) == 0

@@ -1,0 +1,124 @@
+"""GPU parity of the bf16 forward (fa_fwd) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+fa = pytest.importorskip("exact_io_aware_55_b200")
+
+
+def _run_fwd(inp, causal, scale=None, guarded=False):
+    B, H, N, d = inp["shape"]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    q, k, v = (gu.dev_bf16(inp[n + "_bits"]) for n in ("q", "k", "v"))
+    if guarded:
+        og = gu.Guarded((B, H, N, d), torch.bfloat16)
+        lg = gu.Guarded((B, H, N), torch.float32)
+        fa.fa_fwd(q, k, v, og.view, lg.view, scale, causal)
+        torch.cuda.synchronize()
+        assert og.intact() and lg.intact(), "write outside the output buffers"
+        return gu.to_f64(og.view), gu.to_f64(lg.view), scale
+    o, lse = fa.attention_forward(q, k, v, scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    return gu.to_f64(o), gu.to_f64(lse), scale
+
+
+SMALL = [(1, 1, 128, 64), (1, 2, 1, 64), (1, 1, 17, 128), (2, 1, 127, 64), (1, 1, 129, 128),
+         (1, 2, 300, 64), (1, 1, 300, 128), (2, 2, 513, 128), (1, 3, 1000, 64), (1, 1, 640, 128)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SMALL)
+def test_fwd_small_parity(shape, causal):
+    B, H, N, d = shape
+    inp = synth.attention_inputs(B, H, N, d, seed=100 + N + d, with_grad=False)
+    o, lse, scale = _run_fwd(inp, causal, guarded=True)
+    o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], scale, causal)
+    gu.assert_o_lse(o, lse, o_ref, lse_ref, f"{shape} causal={causal}")
+
+
+def test_fwd_pr1_reference_case():
+    """Single head, B=1 H=1 N=128 d=64, fp32 N(0,1) draws rounded to bf16."""
+    inp = synth.attention_inputs_f32_to_bf16(1, 1, 128, 64, seed=1234)
+    o, lse, scale = _run_fwd(inp, False, scale=1.0 / 8.0)
+    o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], scale, False)
+    gu.assert_o_lse(o, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("mult", [8.0, 64.0])
+def test_fwd_large_score_range(mult):
+    """Q scaled by a power of two: frequent running-max moves and rescales."""
+    inp = synth.attention_inputs(1, 2, 1024, 128, seed=77, q_mult=mult, with_grad=False)
+    for causal in (False, True):
+        o, lse, scale = _run_fwd(inp, causal)
+        o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], scale, causal)
+        gu.assert_o_lse(o, lse, o_ref, lse_ref, f"mult={mult} causal={causal}")
+
+
+def test_fwd_config_b4_h16_n2048_d64_full():
+    inp = synth.attention_inputs(4, 16, 2048, 64, seed=1236, with_grad=False)
+    o, lse, scale = _run_fwd(inp, False)
+    o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], scale, False)
+    gu.assert_o_lse(o, lse, o_ref, lse_ref)
+
+
+def _sampled_check(B, H, N, d, causal, seed, q_mult=1.0, n_heads=3, n_rows=24):
+    inp = synth.attention_inputs(B, H, N, d, seed=seed, q_mult=q_mult, with_grad=False, want_f64=False)
+    o, lse, scale = _run_fwd(inp, causal)
+    rng = np.random.default_rng(seed)
+    heads = {(0, 0), (B - 1, H - 1)}
+    while len(heads) < min(n_heads, B * H):
+        heads.add((int(rng.integers(B)), int(rng.integers(H))))
+    for (b, h) in sorted(heads):
+        rows = gu.sample_rows(N, n_rows, seed + 31 * b + h)
+        qh, kh, vh = (synth.head_f64(inp, n, b, h) for n in ("q", "k", "v"))
+        o_ref, lse_ref = oracle.head_forward(qh, kh, vh, scale, causal, rows=rows)
+        gu.assert_o_lse(o[b, h][rows], lse[b, h][rows], o_ref, lse_ref, f"head ({b},{h})")
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+
+
+@pytest.mark.parametrize("q_mult", [1.0, 8.0])
+def test_fwd_config_b2_h16_n8192_d128_causal_sampled(q_mult):
+    _sampled_check(2, 16, 8192, 128, True, seed=1237, q_mult=q_mult)
+
+
+def test_fwd_config_b1_h32_n32768_d128_causal_sampled():
+    _sampled_check(1, 32, 32768, 128, True, seed=1238, n_heads=2, n_rows=16)
+
+
+def test_fwd_noncausal_n8192_d128_sampled():
+    _sampled_check(1, 32, 8192, 128, False, seed=1239, n_heads=2)
+
+
+def test_fwd_empty_and_errors():
+    q = torch.zeros((1, 1, 0, 64), dtype=torch.bfloat16, device="cuda")
+    o, lse = fa.attention_forward(q, q, q)
+    assert o.shape == (1, 1, 0, 64)
+    x = torch.zeros((1, 1, 8, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fa.FAError) as e:
+        fa.attention_forward(x, x, x)
+    assert e.value.status == fa.STATUS_CODES["FA_ERR_UNSUPPORTED"]
+    y = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fa.FAError) as e:
+        fa.attention_forward(y, y, y, scale=-1.0)
+    assert e.value.status == fa.STATUS_CODES["FA_ERR_INVALID_ARG"]
+    assert fa.fa_device_status() == (0, 0)
+
+
+def test_watchdog_selftest_times_out_cleanly():
+    fa.fa_device_status()                      # clear
+    fa.fa_watchdog_selftest(2000)              # 2 ms wait that nobody satisfies
+    st, where = fa.fa_device_status()
+    assert st == fa.STATUS_CODES["FA_ERR_DEVICE_TIMEOUT"] and where == 99
+    assert fa.fa_device_status() == (0, 0)     # cleared, context still usable
+    inp = synth.attention_inputs(1, 1, 64, 64, seed=5, with_grad=False)
+    o, lse, scale = _run_fwd(inp, False)
+    o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], scale, False)
+    gu.assert_o_lse(o, lse, o_ref, lse_ref)
