@@ -111,6 +111,20 @@ class ClockSampler:
 
 
 # -------------------------------------------------------------- our arm
+def apply_shape(args):
+    """--shape/--causal select another workload (profiling runs); the default
+    is the bench workload."""
+    global WORKLOAD_NAME
+    if args.shape:
+        B, H, N, d = (int(x) for x in args.shape.split(","))
+        WORKLOAD.update(B=B, H=H, N=N, d=d)
+    if args.causal:
+        WORKLOAD["causal"] = True
+    if args.shape or args.causal:
+        WORKLOAD_NAME = (f"attention fwd+bwd bf16 B{WORKLOAD['B']} H{WORKLOAD['H']} N{WORKLOAD['N']} "
+                         f"d{WORKLOAD['d']} {'causal' if WORKLOAD['causal'] else 'non-causal'}")
+
+
 def run_ours(args):
     import torch
 
@@ -149,7 +163,7 @@ def run_ours(args):
 
     F = fwd_flops(B, H, N, d, causal)
 
-    def timed(K, W, sampler_window_s=1.5):
+    def timed(K, W, sampler_window_s=args.clock_window):
         for _ in range(W):
             flush.fill_(1.0)
             step()
@@ -423,7 +437,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-step-budget", type=float, default=1.0)
+    ap.add_argument("--shape", default="", help="B,H,N,d of another workload (default: the bench workload)")
+    ap.add_argument("--causal", action="store_true")
+    ap.add_argument("--clock-window", type=float, default=1.5,
+                    help="seconds of steps run under the clock sampler before the timed region")
     args = ap.parse_args()
+    apply_shape(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

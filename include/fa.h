@@ -117,7 +117,7 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
  *   q8, k8, v8 : in,  e4m3 (fn) bytes [B,H,N,d]
  *   o          : out, bf16 [B,H,N,d]
  *   lse        : out, fp32 [B,H,N]
- * d must be 128 or 64; causal is supported.
+ * d must be 128 (a head row is one 128-byte swizzle span); causal is supported.
  */
 FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_descale, float k_descale,
                      float v_descale, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
