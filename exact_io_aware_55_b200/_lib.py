@@ -22,6 +22,7 @@ STATUS_NAMES = {
     5: "FA_ERR_LAUNCH",
     6: "FA_ERR_DEVICE_TIMEOUT",
     7: "FA_ERR_WORKSPACE",
+    8: "FA_ERR_SCRATCH_LIMIT",
 }
 STATUS_CODES = {v: k for k, v in STATUS_NAMES.items()}
 
@@ -49,6 +50,10 @@ def _load() -> ctypes.CDLL:
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_bwd.restype = i
+    lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_bwd_noalloc.restype = i
+    lib.fa_bwd_noalloc_max_bytes.argtypes = []
+    lib.fa_bwd_noalloc_max_bytes.restype = sz
     lib.fa_strerror.argtypes = [i]
     lib.fa_strerror.restype = ctypes.c_char_p
     lib.fa_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]

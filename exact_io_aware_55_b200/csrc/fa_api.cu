@@ -236,6 +236,8 @@ const char* fa_strerror(fa_status s) {
     case FA_ERR_LAUNCH: return "CUDA launch or tensor-map setup failed";
     case FA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
     case FA_ERR_WORKSPACE: return "backward workspace missing or smaller than fa_bwd_workspace_size()";
+    case FA_ERR_SCRATCH_LIMIT:
+      return "shape needs more backward scratch than fa_bwd_noalloc's fixed array (fa_bwd_noalloc_max_bytes())";
   }
   return "unknown fa_status";
 }

@@ -60,7 +60,8 @@ typedef enum fa_status {
   FA_ERR_ARCH = 4,            /* current device is not sm_100 (B200 class) */
   FA_ERR_LAUNCH = 5,          /* CUDA runtime rejected a launch or attribute */
   FA_ERR_DEVICE_TIMEOUT = 6,  /* a bounded device wait ran out (fa_device_status) */
-  FA_ERR_WORKSPACE = 7        /* backward workspace missing or too small */
+  FA_ERR_WORKSPACE = 7,       /* backward workspace missing or too small */
+  FA_ERR_SCRATCH_LIMIT = 8    /* shape needs more than fa_bwd_noalloc's fixed scratch */
 } fa_status;
 
 /*
@@ -122,6 +123,34 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
 FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_descale, float k_descale,
                      float v_descale, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
                      void* stream);
+
+/*
+ * Backward pass for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this is a packaging variant of fa_bwd, not a step of
+ * the method.  Some callers cannot call cudaMalloc where they run the
+ * backward -- a plugin inside a framework that owns every device allocation
+ * and gives the plugin no allocator, or a serving loop that reserves its
+ * memory at start-up and must not allocate (or risk a device-wide
+ * synchronisation) afterwards.  This entry point takes the same arguments as
+ * fa_bwd minus the workspace, and allocates nothing: its scratch is a fixed
+ * array of fa_bwd_noalloc_max_bytes() bytes (64 MiB) inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ *   - Shapes whose fa_bwd_workspace_size() exceeds that limit are rejected
+ *     with FA_ERR_SCRATCH_LIMIT before anything is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; the
+ *     part that must start at zero is cleared by each call itself.  Calls
+ *     whose GPU work overlaps (other streams, unordered host threads) race
+ *     on it and must be serialised by the caller.
+ */
+FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                                float scale, int causal, void* stream);
+
+/* Size in bytes of fa_bwd_noalloc's fixed scratch array. */
+FA_API size_t fa_bwd_noalloc_max_bytes(void);
 
 /* Human-readable text for a status code (static storage, never NULL). */
 FA_API const char* fa_strerror(fa_status status);
