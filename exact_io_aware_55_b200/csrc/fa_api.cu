@@ -107,7 +107,7 @@ fa_status check_shape(int B, int H, int N, int d, float scale, int causal, bool*
   if (!(std::isfinite(scale) && scale > 0.0f)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(B) * H;
-  if (BH > 65535) return FA_ERR_UNSUPPORTED;  // grid.x limit of the launch shape
+  if (BH > 65535) return FA_ERR_UNSUPPORTED;  // grid.y limit of the launch shapes
   // Element offsets are computed in 64-bit; per-head rows in 32-bit.
   if (static_cast<long long>(N) * d > (1ll << 31)) return FA_ERR_UNSUPPORTED;
   *empty = (BH == 0 || N == 0);

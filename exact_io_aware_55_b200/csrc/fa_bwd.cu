@@ -168,8 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int j = blockIdx.y;                          // key tile
+  // Grid: x = key tile (fastest), y = batch-head, so the CTAs resident at any
+  // time cover few heads: their Q/dO tiles and dQ accumulator rows stay in L2.
+  const int bh = blockIdx.y;
+  const int j = blockIdx.x;                          // key tile (0 = heaviest when causal)
   const int N = args.N;
   const int n_q = (N + kTile - 1) / kTile;
   const int i_begin = CAUSAL ? j : 0;
@@ -478,7 +480,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   auto kern = bwd_kernel<D, CAUSAL>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(a.BH, (a.N + kTile - 1) / kTile);
+  dim3 grid((a.N + kTile - 1) / kTile, a.BH);
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

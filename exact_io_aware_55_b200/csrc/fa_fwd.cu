@@ -38,6 +38,12 @@ constexpr int kBN = 128;        // key rows per K/V tile
 constexpr int kNQT = 2;         // Q tiles per CTA
 constexpr int kThreads = 384;   // 12 warps
 constexpr float kRescaleThresh = 8.0f;
+// Registers per thread after re-balancing: warpgroup 0 (producer, MMA, two
+// idle warps) gives registers to the two softmax warpgroups.  Launch: 384
+// threads x 168 = 64512; after: 128 x 64 + 256 x 216 = 63488.
+constexpr uint32_t kRegsWG0 = 64;
+constexpr uint32_t kRegsSoftmax = 216;
+static_assert(128 * kRegsWG0 + 256 * kRegsSoftmax <= 384 * 168, "register split exceeds the launch allocation");
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D, bool FP8>
@@ -51,6 +57,10 @@ struct FwdShape {
   static constexpr int kSSteps = kRowBytes / 32;            // MMA K-steps of S = Q K^T (32 B each)
   static constexpr int kPVRows = FP8 ? 32 : 16;             // keys per PV MMA step
   static constexpr int kPVSteps = kBN / kPVRows;
+  // Exponentials per 8 on the FMA pipe (exp2_fma2) instead of MUFU, on tiles
+  // without masked entries: where the MMA time per tile is shorter (d = 64,
+  // e4m3) the MUFU unit alone would bound the kernel, so more is moved.
+  static constexpr int kEmuPer8 = (D == 64 || FP8) ? 3 : 1;
   static constexpr uint32_t kIdS = FP8 ? idesc_e4m3(128, 128, false, false) : idesc_bf16(128, 128, false, false);
   static constexpr uint32_t kIdPV = FP8 ? idesc_e4m3(128, D, false, true) : idesc_bf16(128, D, false, true);
   static_assert(kRowBytes % 128 == 0, "head row must be a whole number of 128-byte chunks");
@@ -75,6 +85,54 @@ constexpr size_t fwd_smem_bytes() {
   return 1024 /*alignment slack*/ + size_t(kNQT + 2 * S::kNST) * S::kTileBytes + sizeof(FwdBarriers<S::kNST>);
 }
 
+// Row maximum of 128 scores: four independent chains of 3-input max.
+__device__ __forceinline__ float row_max128(const float (&sv)[128]) {
+  float acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float a = sv[32 * k];
+#pragma unroll
+    for (int t = 1; t + 1 < 32; t += 2) a = fmax3(a, sv[32 * k + t], sv[32 * k + t + 1]);
+    acc[k] = fmaxf(a, sv[32 * k + 31]);
+  }
+  return fmax3(acc[0], acc[1], fmaxf(acc[2], acc[3]));
+}
+
+// p = 2^(s*c - m) for 128 scores; packs P for the PV MMA (bf16 pairs or e4m3
+// quads) and returns the fp32 row sum of p.  EMU of every 8 pairs (bf16) or
+// quads (e4m3) use the FMA-pipe exponential, the rest MUFU ex2.
+template <bool FP8, int EMU>
+__device__ __forceinline__ float row_exp128(const float (&sv)[128], float c, float neg_m,
+                                            uint32_t (&pk)[FP8 ? 32 : 64]) {
+  const float2 cc = make_float2(c, c), nm = make_float2(neg_m, neg_m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  auto ex = [&](float2 x, bool emu) {
+    return emu ? exp2_fma2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+  };
+  if constexpr (!FP8) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      const float2 x = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), cc, nm);
+      const float2 p = ex(x, (i & 7) < EMU);
+      acc[i & 3] = fadd2(acc[i & 3], p);
+      pk[i] = pack_bf16x2(p.x, p.y);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const bool emu = (i & 7) < EMU;
+      const float2 pa = ex(ffma2(make_float2(sv[4 * i], sv[4 * i + 1]), cc, nm), emu);
+      const float2 pb = ex(ffma2(make_float2(sv[4 * i + 2], sv[4 * i + 3]), cc, nm), emu);
+      acc[(2 * i) & 3] = fadd2(acc[(2 * i) & 3], pa);
+      acc[(2 * i + 1) & 3] = fadd2(acc[(2 * i + 1) & 3], pb);
+      pk[i] = pack_e4m3x4(pa.x, pa.y, pb.x, pb.y);
+    }
+  }
+  const float2 s01 = fadd2(acc[0], acc[1]), s23 = fadd2(acc[2], acc[3]);
+  const float2 s = fadd2(s01, s23);
+  return s.x + s.y;
+}
+
 template <int D, bool CAUSAL, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -91,9 +149,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  // Causal: heaviest Q-tile pairs first (block rows are scheduled in order).
-  const int pair = CAUSAL ? int(gridDim.y - 1 - blockIdx.y) : int(blockIdx.y);
+  // Grid: x = Q-tile pair (fastest), y = batch-head, so the CTAs resident at
+  // any time cover few heads and their K/V tiles are re-read from L2, not HBM.
+  // Causal: heaviest pairs of each head first.
+  const int bh = blockIdx.y;
+  const int pair = CAUSAL ? int(gridDim.x - 1 - blockIdx.x) : int(blockIdx.x);
   const int N = args.N;
   const int n_kv = (N + kBN - 1) / kBN;
 
@@ -130,6 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  if (warp < 4) {
+    regs_dec<kRegsWG0>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -236,20 +298,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           (void)mbar_wait(&bars->kv_empty[(Tmax - 1) % NST], ((Tmax - 1) / NST) & 1, wc, WAIT_FWD_KV_EMPTY);
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------- softmax
     const int g = (warp - 4) >> 2;
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;
-    const int qrow = q0[g] + row;
+    const int q0g = pair * (kNQT * kBM) + g * kBM;
+    const int Tg = (q0g < N) ? (CAUSAL ? min(n_kv, q0g / kBN + 1) : n_kv) : 0;
+    const int qrow = q0g + row;
     const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
     const uint32_t s_tmem = lane_base + uint32_t(g * 128);
     const uint32_t o_tmem = lane_base + uint32_t(kNQT * 128 + g * D);
     const float c = args.c_log2;
     float m_ref = -INFINITY;
     float l = 0.0f;
-    bool ok = T[g] > 0;
-    for (int j = 0; j < T[g]; ++j) {
+    bool ok = Tg > 0;
+    for (int j = 0; j < Tg; ++j) {
       if (!mbar_wait_warp(&bars->s_full[g], j & 1, wc, WAIT_FWD_S)) {
         ok = false;
         break;
@@ -264,17 +330,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; ++i) sv[q * 32 + i] = __uint_as_float(r[i]);
       }
       const int k0 = j * kBN;
-      const bool need_mask = (k0 + kBN > N) || (CAUSAL && k0 + kBN - 1 > q0[g]);
+      const bool need_mask = (k0 + kBN > N) || (CAUSAL && k0 + kBN - 1 > q0g);
       if (need_mask) {
         const int lim = CAUSAL ? min(N - 1, qrow) : (N - 1);   // last visible key
 #pragma unroll
         for (int i = 0; i < 128; ++i)
           if (k0 + i > lim) sv[i] = -INFINITY;
       }
-      float mx = sv[0];
-#pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
-      const float m_tile = mx * c;
+      const float m_tile = row_max128(sv) * c;
       float alpha = 1.0f;
       bool rescale = false;
       if (j == 0) {
@@ -285,36 +348,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         rescale = true;
       }
       const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
-      float rs0 = 0.0f, rs1 = 0.0f;
+      float row_sum;
       if constexpr (!FP8) {
         uint32_t pk[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2_approx(fmaf(sv[2 * i], c, neg_m));
-          const float p1 = ex2_approx(fmaf(sv[2 * i + 1], c, neg_m));
-          rs0 += p0;
-          rs1 += p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
+        row_sum = need_mask ? row_exp128<false, 0>(sv, c, neg_m, pk)
+                            : row_exp128<false, S::kEmuPer8>(sv, c, neg_m, pk);
         uint32_t (&pa)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
         uint32_t (&pb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
         tmem_st_x32(s_tmem, pa);
         tmem_st_x32(s_tmem + 32, pb);
       } else {
         uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(sv[4 * i], c, neg_m));
-          const float p1 = ex2_approx(fmaf(sv[4 * i + 1], c, neg_m));
-          const float p2 = ex2_approx(fmaf(sv[4 * i + 2], c, neg_m));
-          const float p3 = ex2_approx(fmaf(sv[4 * i + 3], c, neg_m));
-          rs0 += p0 + p2;
-          rs1 += p1 + p3;
-          pk[i] = pack_e4m3x4(p0, p1, p2, p3);
-        }
+        row_sum = need_mask ? row_exp128<true, 0>(sv, c, neg_m, pk)
+                            : row_exp128<true, S::kEmuPer8>(sv, c, neg_m, pk);
         tmem_st_x32(s_tmem, pk);
       }
-      l = l * alpha + (rs0 + rs1);
+      l = l * alpha + row_sum;
       if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
@@ -369,7 +418,7 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   auto kern = fwd_kernel<D, CAUSAL, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(a.BH, (a.N + kNQT * kBM - 1) / (kNQT * kBM));
+  dim3 grid((a.N + kNQT * kBM - 1) / (kNQT * kBM), a.BH);
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }

@@ -288,6 +288,18 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[
                : "memory");
 }
 
+// Per-warpgroup register re-balancing; every warp of the warpgroup executes it.
+// The counts a kernel uses must add up, over its warpgroups, to no more than
+// the registers the block was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -299,6 +311,64 @@ __device__ __forceinline__ float lg2_approx(float x) {
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pairs (one f32x2 instruction for two lanes of work).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for a pair of finite or -inf arguments <= 2^22, on the FMA pipe instead
+// of the MUFU unit.  Range reduction x = n + f, n = round-to-nearest(x) taken
+// by adding 1.5 * 2^23 (the integer lands in the low mantissa bits), |f| <= 1/2;
+// 2^f by a degree-3 polynomial fitted for minimax relative error on [-1/2, 1/2]
+// (coefficients from gen_exp2_poly.py: max relative error 8.3e-5 = 2^-13.5);
+// 2^n by adding n to the exponent field.  Arguments below -120 are clamped to
+// -120, so the result is then about 7.5e-37 instead of 0: callers use it only
+// where no argument is masked to -inf.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+  x.x = fmaxf(x.x, -120.0f);
+  x.y = fmaxf(x.y, -120.0f);
+  const float2 t = fadd2(x, make_float2(kMagic, kMagic));
+  const float2 j = fadd2(t, make_float2(-kMagic, -kMagic));
+  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), x);   // x - n, exact
+  float2 p = ffma2(make_float2(5.521299317e-02f, 5.521299317e-02f), f,
+                   make_float2(2.427141368e-01f, 2.427141368e-01f));
+  p = ffma2(p, f, make_float2(6.932621598e-01f, 6.932621598e-01f));
+  p = ffma2(p, f, make_float2(9.999195933e-01f, 9.999195933e-01f));
+  return make_float2(__uint_as_float((__float_as_uint(t.x) << 23) + __float_as_uint(p.x)),
+                     __uint_as_float((__float_as_uint(t.y) << 23) + __float_as_uint(p.y)));
+}
+
 // Two floats -> packed bf16x2 (lo in bits 0..15), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
