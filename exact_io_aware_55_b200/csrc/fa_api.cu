@@ -215,8 +215,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
-  a.dvec = reinterpret_cast<float*>(ws + wl.dvec_off);
-  a.lse2 = reinterpret_cast<float*>(ws + wl.lse2_off);
+  a.neg_dvec = reinterpret_cast<float*>(ws + wl.dvec_off);
+  a.neg_lse2 = reinterpret_cast<float*>(ws + wl.lse2_off);
   a.dq_acc = reinterpret_cast<float*>(ws + wl.dq_off);
   a.N = N;
   a.Np = static_cast<int>(padded_rows(N));

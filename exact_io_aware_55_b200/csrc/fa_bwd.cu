@@ -10,7 +10,7 @@
 //   dQ = scale dS K, dK = scale dS^T Q.
 //
 // Three launches on the caller's stream:
-//   bwd_pre      D and LSE*log2(e) per row (padded to 128-row tiles, +inf LSE on
+//   bwd_pre      -D and -LSE*log2(e) per row (padded to 128-row tiles, -inf on
 //                padding rows so their P is exactly 0) and zeroing of the fp32
 //                dQ accumulator.
 //   bwd_kernel   one CTA per (key tile j, batch-head); K_j, V_j stay in shared
@@ -22,13 +22,16 @@
 //                  dV_j += P^T dO_i     (A = P^T from TMEM)
 //                  dS^T = scale P^T o (dP^T - D_i) -> shared memory (bf16, swizzled)
 //                  dK_j += dS^T Q_i     (A = dS^T, K-major)
-//                  dQ_i  = dS K_j       -> TMEM R2 (A = the same dS^T bytes read
-//                                          MN-major), then fp32 red.add into the
-//                                          workspace accumulator
+//                  dQ_i^T = K_j^T dS^T  -> TMEM R2 (both operands read MN-major
+//                                          from the K tile and the dS^T bytes),
+//                                          then fp32 red.add into the workspace
+//                                          accumulator, one d-contiguous line per
+//                                          query row
 //   bwd_dq_final dQ accumulator -> bf16.
 // Warp roles in bwd_kernel: 0 TMA producer, 1 MMA issuer (+TMEM owner),
-// 4-7 the P / dS warpgroup (thread = key row = TMEM lane), 8-11 the dQ
-// warpgroup (thread = query row).  Epilogue: warps 4-7 store dV, 8-11 dK.
+// 4-7 and 8-11 the two P / dS warpgroups (thread = key row = TMEM lane; each
+// handles 64 of the 128 queries of a tile), 12-15 the dQ warpgroup (thread =
+// d index of dQ^T).  Epilogue: warps 4-7 store dV, 8-11 dK.
 // TMEM columns: dV [0,d) dK [d,2d) R1 [2d,2d+128) R2 [2d+128,2d+256).
 #include <cuda_bf16.h>
 
@@ -40,8 +43,15 @@ namespace fa {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr float kLog2e = 1.4426950408889634f;
+// Registers per thread after re-balancing.  Launch: 512 threads x 128 = 65536;
+// after: warpgroup 0 (producer, MMA, 2 idle warps) 80, the two P/dS
+// warpgroups 144, the dQ warpgroup 144: 128 x (80 + 2 x 144 + 144) = 65536.
+constexpr uint32_t kRegsWG0 = 80;
+constexpr uint32_t kRegsPdS = 144;
+constexpr uint32_t kRegsDQ = 144;
+static_assert(128 * (kRegsWG0 + 2 * kRegsPdS + kRegsDQ) <= 512 * 128, "register split exceeds the launch allocation");
 
 // ------------------------------------------------------------- preprocess
 template <int D>
@@ -73,8 +83,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a, int row_blocks,
     for (int m = TPR / 2; m > 0; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
     if (sub == 0 && in_range) {
       const size_t r = size_t(bh) * a.Np + i;
-      a.dvec[r] = (i < a.N) ? part : 0.0f;
-      a.lse2[r] = (i < a.N) ? a.lse[size_t(bh) * a.N + i] * kLog2e : INFINITY;
+      a.neg_dvec[r] = (i < a.N) ? -part : 0.0f;
+      a.neg_lse2[r] = (i < a.N) ? -a.lse[size_t(bh) * a.N + i] * kLog2e : -INFINITY;
     }
   } else {
     const long long stride = (long long)(gridDim.x - row_blocks) * blockDim.x;
@@ -111,8 +121,12 @@ struct BwdShape {
   static constexpr int kKSteps = kRowBytes / 32;         // K-steps over d (16 elements)
   static constexpr uint32_t kIdSS = idesc_bf16(128, 128, false, false);   // S^T, dP^T
   static constexpr uint32_t kIdKmaj = idesc_bf16(128, D, false, true);    // dV, dK: B MN-major
-  static constexpr uint32_t kIdDQ = idesc_bf16(128, D, true, true);       // dQ: A and B MN-major
+  // dQ^T = K^T dS^T: M = d (key-tile rows become TMEM lanes = d), N = 128
+  // queries, both operands MN-major (the K tile and the dS^T buffer as stored).
+  static constexpr uint32_t kIdDQT = idesc_bf16(D, 128, true, true);
   static constexpr uint32_t kColDV = 0, kColDK = D, kColR1 = 2 * D, kColR2 = 2 * D + 128;
+  // Exponentials per 8 pairs computed on the FMA pipe on fully unmasked tiles.
+  static constexpr int kEmuPer8 = (D == 64) ? 3 : 2;
 };
 
 template <int NST>
@@ -131,9 +145,8 @@ constexpr size_t bwd_smem_bytes() {
   return size_t(2 + 2 * S::kNST) * S::kTileBytes + S::kDsBytes + S::kNST * 1024 + sizeof(BwdBarriers<S::kNST>);
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
+__device__ __forceinline__ void red_add_f32(float* addr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -181,12 +194,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bars->qdo_full[s], 1);
-      mbar_init(&bars->qdo_empty[s], 1 + 4);
+      mbar_init(&bars->qdo_empty[s], 1 + 8);
     }
     mbar_init(&bars->s_ready, 1);
     mbar_init(&bars->dp_ready, 1);
-    mbar_init(&bars->p_ready, 4);
-    mbar_init(&bars->ds_ready, 4);
+    mbar_init(&bars->p_ready, 8);
+    mbar_init(&bars->ds_ready, 8);
     mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dq_ready, 1);
     mbar_init(&bars->dq_free, 4);
@@ -203,6 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  if (warp < 4) {
+    regs_dec<kRegsWG0>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -231,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                            bh, pol_q);
         }
         const size_t srow = size_t(bh) * args.Np + size_t(i) * kTile;
-        bulk_load(sStat + s * 256, args.lse2 + srow, 512, &bars->qdo_full[s]);
-        bulk_load(sStat + s * 256 + 128, args.dvec + srow, 512, &bars->qdo_full[s]);
+        bulk_load(sStat + s * 256, args.neg_lse2 + srow, 512, &bars->qdo_full[s]);
+        bulk_load(sStat + s * 256 + 128, args.neg_dvec + srow, 512, &bars->qdo_full[s]);
       }
     }
   } else if (warp == 1) {
@@ -268,9 +283,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           // dV += P^T dO: A = P^T (TMEM R1, bf16), B = dO MN-major; 16 queries per step.
 #pragma unroll
+          // P^T of queries 0-63 sits in R1 columns [0,32), of queries 64-127 in [96,128).
           for (int kt = 0; kt < 8; ++kt)
-            mma_f16_ts(tmem + S::kColDV, tR1 + kt * 8, sdesc_sw128(doa + kt * 2048, 16384, 1024), S::kIdKmaj,
-                       (it > 0 || kt > 0) ? 1u : 0u);
+            mma_f16_ts(tmem + S::kColDV, tR1 + kt * 8 + (kt >= 4 ? 64 : 0), sdesc_sw128(doa + kt * 2048, 16384, 1024),
+                       S::kIdKmaj, (it > 0 || kt > 0) ? 1u : 0u);
           if (it + 1 < n_iter) {                        // S^T of the next query tile
             const int sn = (it + 1) % NST;
             if (!mbar_wait(&bars->qdo_full[sn], ((it + 1) / NST) & 1, wc, WAIT_BWD_QDO)) { ok = false; break; }
@@ -287,11 +303,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16_ss(tmem + S::kColDK, sdesc_sw128(sdSa + off, 16, 1024),
                        sdesc_sw128(qa + kt * 2048, 16384, 1024), S::kIdKmaj, (it > 0 || kt > 0) ? 1u : 0u);
           }
-          // dQ = dS K: A = the dS^T bytes read MN-major (M = queries), B = K MN-major; 16 keys per step.
+          // dQ^T = K^T dS^T: A = K read MN-major (M = d), B = the dS^T bytes read
+          // MN-major (N = queries); 16 keys per step.  The transposed product puts
+          // d on the TMEM lanes, so each dQ row update is one coalesced line.
 #pragma unroll
           for (int kt = 0; kt < 8; ++kt)
-            mma_f16_ss(tR2, sdesc_sw128(sdSa + kt * 2048, 16384, 1024), sdesc_sw128(sKa + kt * 2048, 16384, 1024),
-                       S::kIdDQ, kt > 0 ? 1u : 0u);
+            mma_f16_ss(tR2, sdesc_sw128(sKa + kt * 2048, 16384, 1024), sdesc_sw128(sdSa + kt * 2048, 16384, 1024),
+                       S::kIdDQT, kt > 0 ? 1u : 0u);
           tc_commit(&bars->dq_ready);
           tc_commit(&bars->ds_free);
           tc_commit(&bars->qdo_empty[s]);
@@ -300,49 +318,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) (void)mbar_wait(&bars->final_, 0, wc, WAIT_BWD_FINAL);
       }
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------- P / dS group
+  }
+  } else if (warp < 12) {
+    regs_inc<kRegsPdS>();
+    // --------------------------------------------------- P / dS groups
+    // Two warpgroups; group h handles queries [64h, 64h+64) of every tile.
+    const int h = (warp - 4) >> 2;
     const int wq = warp & 3;
     const int c = wq * 32 + lane;                   // key row within the tile
     const int kv = j * kTile + c;
     const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
-    const uint32_t tR1 = lane_base + S::kColR1, tR2 = lane_base + S::kColR2;
+    const uint32_t tS = lane_base + S::kColR1 + 64 * h;        // this half's S^T columns
+    const uint32_t tP = lane_base + S::kColR1 + 96 * h;        // its P^T (bf16) columns
+    const uint32_t tdP = lane_base + S::kColR2 + 64 * h;       // this half's dP^T columns
     const float cl = args.c_log2;
     const float scale = args.scale;
     const bool kv_valid = kv < N;
+    const bool kv_tile_full = (j + 1) * kTile <= N;
+    uint8_t* ds_row = sdS + h * 16384 + (c >> 3) * 1024 + (c & 7) * 128;
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       const int s = it % NST;
       const int i = i_begin + it;
-      const float* sl = sStat + s * 256;            // lse2 of the 128 queries
-      const float* sd = sl + 128;                   // D of the 128 queries
-      // LSE2 / D of this stage arrived by bulk copy on qdo_full; S^T by MMA commit.
+      const float* snl = sStat + s * 256 + 64 * h;   // -LSE2 of this half's queries
+      const float* snd = snl + 128;                  // -D of this half's queries
+      // -LSE2 / -D of this stage arrived by bulk copy on qdo_full; S^T by MMA commit.
       if (!mbar_wait_warp(&bars->qdo_full[s], (it / NST) & 1, wc, WAIT_BWD_QDO)) { ok = false; break; }
       if (!mbar_wait_warp(&bars->s_ready, it & 1, wc, WAIT_BWD_S)) { ok = false; break; }
       tc_fence_after();
-      // P^T row: exp2(S^T * scale * log2e - LSE2_q); masked entries are 0.
+      // P^T = exp2(S^T * scale * log2e - LSE2_q); masked and padded entries are 0.
       const bool diag = CAUSAL && (i == j);
-      uint32_t pk[64];
+      const bool exact = diag || !kv_tile_full || (i + 1) * kTile > N;
+      uint32_t pk[32];
+      {
+        uint32_t r[64];
+        tmem_ld_x64(tS, r);
+        const float2 cc = make_float2(cl, cl);
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t r[32];
-        tmem_ld_x32(tR1 + q4 * 32, r);
-        uint32_t w[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int q0 = q4 * 32 + 2 * t;
-          float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * t]), cl, -sl[q0]));
-          float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * t + 1]), cl, -sl[q0 + 1]));
-          if (diag) {
-            if (c > q0) p0 = 0.0f;
-            if (c > q0 + 1) p1 = 0.0f;
+        for (int t = 0; t < 32; ++t) {
+          const float2 nl = *reinterpret_cast<const float2*>(snl + 2 * t);
+          const float2 x = ffma2(make_float2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1])), cc, nl);
+          float2 p;
+          if (!exact && (t & 7) < S::kEmuPer8) {
+            p = exp2_fma2(x);
+          } else {
+            p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (diag) {
+              const int q0 = 64 * h + 2 * t;
+              if (c > q0) p.x = 0.0f;
+              if (c > q0 + 1) p.y = 0.0f;
+            }
+            if (!kv_valid) p = make_float2(0.0f, 0.0f);
           }
-          if (!kv_valid) p0 = p1 = 0.0f;
-          w[t] = pack_bf16x2(p0, p1);
-          pk[q4 * 16 + t] = w[t];
+          pk[t] = pack_bf16x2(p.x, p.y);
         }
-        tmem_st_x16(tR1 + q4 * 16, w);
       }
+      tmem_st_x32(tP, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -351,45 +382,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_warp(&bars->dp_ready, it & 1, wc, WAIT_BWD_DP)) { ok = false; break; }
       if (it > 0 && !mbar_wait_warp(&bars->ds_free, (it - 1) & 1, wc, WAIT_BWD_DS_FREE)) { ok = false; break; }
       tc_fence_after();
-      uint8_t* row_base = sdS + (c >> 3) * 1024 + (c & 7) * 128;
+      {
+        uint32_t r[64];
+        tmem_ld_x64(tdP, r);
+        const float2 sc2 = make_float2(scale, scale);
+        uint32_t w[32];
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t r[32];
-        tmem_ld_x32(tR2 + q4 * 32, r);
-        uint32_t w[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int q0 = q4 * 32 + 2 * t;
-          const uint32_t pw = pk[q4 * 16 + t];
-          const float ds0 = scale * bf16lo(pw) * (__uint_as_float(r[2 * t]) - sd[q0]);
-          const float ds1 = scale * bf16hi(pw) * (__uint_as_float(r[2 * t + 1]) - sd[q0 + 1]);
-          w[t] = pack_bf16x2(ds0, ds1);
+        for (int t = 0; t < 32; ++t) {
+          const float2 nd = *reinterpret_cast<const float2*>(snd + 2 * t);
+          const float2 dpm = fadd2(make_float2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1])), nd);
+          const float2 ps = fmul2(make_float2(bf16lo(pk[t]), bf16hi(pk[t])), sc2);
+          const float2 ds = fmul2(ps, dpm);
+          w[t] = pack_bf16x2(ds.x, ds.y);
         }
-        // 32 queries = 64 bytes = four 16-byte units of chunk (q4 >> 1).
-        uint8_t* chunk = row_base + (q4 >> 1) * 16384;
+        // 64 queries = 128 bytes = one full row of chunk h, eight 16-byte units.
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = (q4 & 1) * 4 + u;
-          *reinterpret_cast<uint4*>(chunk + ((unit ^ (c & 7)) << 4)) =
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(ds_row + ((u ^ (c & 7)) << 4)) =
               make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bars->ds_ready);
-        mbar_arrive(&bars->qdo_empty[s]);           // done with this stage's LSE2 / D
+        mbar_arrive(&bars->qdo_empty[s]);           // done with this stage's -LSE2 / -D
       }
     }
-    // dV epilogue
+    // Epilogue: group 0 stores dV, group 1 stores dK.
     if (ok && mbar_wait_warp(&bars->final_, 0, wc, WAIT_BWD_FINAL)) {
       tc_fence_after();
-      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.dv) + (size_t(bh) * N + kv) * D;
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(h == 0 ? args.dv : args.dk) + (size_t(bh) * N + kv) * D;
+      const uint32_t src = lane_base + (h == 0 ? S::kColDV : S::kColDK);
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         uint32_t r[32];
-        tmem_ld_x32(lane_base + S::kColDV + q * 32, r);
+        tmem_ld_x32(src + q * 32, r);
         if (kv_valid) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -403,54 +431,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp >= 8) {
+  } else {
+    regs_inc<kRegsDQ>();
     // ---------------------------------------------------------- dQ group
+    // dQ^T tile in TMEM R2: lane = d index, column = query.  With M = d = 128
+    // every lane of the warp's quarter holds a d row; with M = 64 the rows sit
+    // in the first 16 lanes of each quarter (row m -> lane m % 16 + 32 (m / 16)).
     const int wq = warp & 3;
-    const int r0 = wq * 32 + lane;                  // query row within the tile (dQ) / key row (dK)
     const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
+    const int dcol = (D == 128) ? (wq * 32 + lane) : (wq * 16 + lane);
+    const bool dcol_valid = (D == 128) || (lane < 16);
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int i = i_begin + it;
       if (!mbar_wait_warp(&bars->dq_ready, it & 1, wc, WAIT_BWD_DQ)) { ok = false; break; }
       tc_fence_after();
-      float dq[D];
-#pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t r[32];
-        tmem_ld_x32(lane_base + S::kColR2 + q * 32, r);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) dq[q * 32 + t] = __uint_as_float(r[t]);
-      }
+      uint32_t dqt[128];
+      tmem_ld_x64(lane_base + S::kColR2, *reinterpret_cast<uint32_t(*)[64]>(&dqt[0]));
+      tmem_ld_x64(lane_base + S::kColR2 + 64, *reinterpret_cast<uint32_t(*)[64]>(&dqt[64]));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dq_free);
-      const int qrow = i * kTile + r0;
-      if (qrow < N) {
-        float* dst = args.dq_acc + (size_t(bh) * N + qrow) * D;
+      // One query row per instruction: the warp's lanes cover consecutive d.
+      float* base = args.dq_acc + (size_t(bh) * N + size_t(i) * kTile) * D + dcol;
+      const int rows = min(kTile, N - i * kTile);
+      if (dcol_valid) {
 #pragma unroll
-        for (int t = 0; t < D / 4; ++t) red_add_v4(dst + 4 * t, dq[4 * t], dq[4 * t + 1], dq[4 * t + 2], dq[4 * t + 3]);
-      }
-    }
-    // dK epilogue
-    if (ok && mbar_wait_warp(&bars->final_, 0, wc, WAIT_BWD_FINAL)) {
-      tc_fence_after();
-      const int kv = j * kTile + r0;
-      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.dk) + (size_t(bh) * N + kv) * D;
-#pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t r[32];
-        tmem_ld_x32(lane_base + S::kColDK + q * 32, r);
-        if (kv < N) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]), __uint_as_float(r[8 * u + 1]));
-            v.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]), __uint_as_float(r[8 * u + 3]));
-            v.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]), __uint_as_float(r[8 * u + 5]));
-            v.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]), __uint_as_float(r[8 * u + 7]));
-            reinterpret_cast<uint4*>(dst + q * 32)[u] = v;
-          }
-        }
+        for (int q = 0; q < 128; ++q)
+          if (q < rows) red_add_f32(base + size_t(q) * D, __uint_as_float(dqt[q]));
       }
     }
   }

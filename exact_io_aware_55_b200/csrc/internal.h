@@ -48,8 +48,8 @@ struct BwdArgs {
   void* dq;           // bf16 [BH, N, d]
   void* dk;           // bf16 [BH, N, d]
   void* dv;           // bf16 [BH, N, d]
-  float* dvec;        // workspace: D, fp32 [BH, Np]
-  float* lse2;        // workspace: LSE * log2(e), fp32 [BH, Np] (+inf on padded rows)
+  float* neg_dvec;    // workspace: -D, fp32 [BH, Np] (0 on padded rows)
+  float* neg_lse2;    // workspace: -LSE * log2(e), fp32 [BH, Np] (-inf on padded rows)
   float* dq_acc;      // workspace: fp32 [BH, N, d]
   int N;
   int Np;             // N rounded up to a multiple of 128
