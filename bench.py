@@ -130,6 +130,7 @@ def run_ours(args):
 
     import exact_io_aware_55_b200 as fa
     import synth
+    from exact_io_aware_55_b200.dist import max_over_ranks
 
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -205,11 +206,7 @@ def run_ours(args):
     if st != 0:
         raise RuntimeError(f"device status {st} (wait site {where}) during the bench")
 
-    t_step = t_fwd + t_bwd
-    if dist is not None:
-        tt = torch.tensor([t_step, t_fwd, t_bwd], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step, t_fwd, t_bwd = (float(x) for x in tt.tolist())
+    t_step, t_fwd, t_bwd = max_over_ranks(dist, [t_fwd + t_bwd, t_fwd, t_bwd], dev)
     value = ws * 3.5 * F / (t_step * 1e-3) / 1e12
     fwd_tflops = ws * F / (t_fwd * 1e-3) / 1e12
     bwd_tflops = ws * 2.5 * F / (t_bwd * 1e-3) / 1e12
@@ -242,11 +239,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    t_e2e = e0.elapsed_time(e1) / K2
-    if dist is not None:
-        tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_e2e = float(tt.item())
+    t_e2e = max_over_ranks(dist, [e0.elapsed_time(e1) / K2], dev)[0]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
 
@@ -263,7 +256,7 @@ def run_ours(args):
             "peak_source": f"{peak_src} bf16_tflops (burst; each launch is timed alone)"}
 
     if rank == 0:
-        cpu = cpu_baseline(args) if ws >= 1 and not args.no_cpu_baseline and ws == 1 else None
+        cpu = cpu_baseline(args) if (ws == 1 and not args.no_cpu_baseline) else None
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True, "scaling": "weak",

@@ -1,0 +1,91 @@
+"""The C ABI without a GPU: every symbol declared in include/fa.h is exported
+by libfa.so, and argument errors come back as status codes before anything
+touches a device (so these calls are safe on any host)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_io_aware_55_b200 as fa
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "fa.h")
+F = ctypes.c_float
+C = fa.STATUS_CODES
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text, flags=re.M)
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert {"fa_fwd", "fa_bwd", "fa_fwd_fp8", "fa_bwd_workspace_size", "fa_strerror"} <= set(names)
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_texts():
+    assert fa.strerror(0) == "ok"
+    for code in range(1, 9):
+        assert len(fa.strerror(code)) > 5
+    assert "unknown" in fa.strerror(99)
+    assert fa.lib.fa_version() >= 100
+
+
+def test_workspace_size_formula():
+    # rows padded to 128: (-D, -LSE2) fp32, each rounded up to 256 B, then the fp32 dQ accumulator
+    def expect(B, H, N, d):
+        rows = B * H * ((N + 127) // 128 * 128)
+        stat = (rows * 4 + 255) // 256 * 256
+        return 2 * stat + B * H * N * d * 4
+    for shape in [(1, 1, 128, 64), (2, 3, 1000, 128), (4, 16, 2048, 64), (1, 1, 1, 64)]:
+        assert fa.fa_bwd_workspace_size(*shape) == expect(*shape)
+    assert fa.fa_bwd_workspace_size(1, 1, 0, 64) == 0
+    with pytest.raises(fa.FAError):
+        fa.fa_bwd_workspace_size(1, 1, 16, 96)
+    assert fa.lib.fa_bwd_workspace_size(-1, 1, 16, 64) == ctypes.c_size_t(-1).value
+
+
+def fwd(q, o, lse, B=1, H=1, N=128, d=64, scale=0.125, causal=0):
+    return fa.lib.fa_fwd(q, q, q, o, lse, B, H, N, d, F(scale), causal, None)
+
+
+def test_forward_argument_errors_launch_nothing():
+    assert fwd(None, None, None) == C["FA_ERR_INVALID_ARG"]
+    assert fwd(4096, 4096, 4096, d=96) == C["FA_ERR_UNSUPPORTED"]
+    assert fwd(4096, 4096, 4096, scale=0.0) == C["FA_ERR_INVALID_ARG"]
+    assert fwd(4096, 4096, 4096, scale=float("nan")) == C["FA_ERR_INVALID_ARG"]
+    assert fwd(4096, 4096, 4096, causal=2) == C["FA_ERR_INVALID_ARG"]
+    assert fwd(4096, 4096, 4096, N=-5) == C["FA_ERR_INVALID_ARG"]
+    assert fwd(4104, 4096, 4096) == C["FA_ERR_ALIGNMENT"]          # 8-byte aligned only
+    assert fwd(4096, 4096, 4098) == C["FA_ERR_ALIGNMENT"]          # lse needs 4 bytes
+    assert fwd(None, None, None, N=0) == C["FA_OK"]                # empty: nothing to do
+    assert fwd(None, None, None, B=0) == C["FA_OK"]
+    assert fa.lib.fa_fwd_fp8(4096, 4096, 4096, F(1), F(1), F(1), 4096, 4096, 1, 1, 16, 64, F(0.1), 0,
+                             None) == C["FA_ERR_UNSUPPORTED"]         # e4m3 path needs d = 128
+    assert fa.lib.fa_fwd_fp8(4096, 4096, 4096, F(0), F(1), F(1), 4096, 4096, 1, 1, 16, 128, F(0.1), 0,
+                             None) == C["FA_ERR_INVALID_ARG"]
+
+
+def test_backward_argument_errors_launch_nothing():
+    p = 4096
+    args = [p] * 6 + [p] * 3
+    assert fa.lib.fa_bwd(*args, 1, 1, 64, 64, F(0.125), 0, None, 0, None) == C["FA_ERR_WORKSPACE"]
+    assert fa.lib.fa_bwd(*args, 1, 1, 64, 64, F(0.125), 0, p, 16, None) == C["FA_ERR_WORKSPACE"]
+    need = fa.fa_bwd_workspace_size(1, 1, 64, 64)
+    assert fa.lib.fa_bwd(*([p] * 5 + [p + 2] + [p] * 3), 1, 1, 64, 64, F(0.125), 0, p, need,
+                         None) == C["FA_ERR_ALIGNMENT"]
+    assert fa.lib.fa_bwd(*([None] + [p] * 8), 1, 1, 64, 64, F(0.125), 0, p, need, None) == C["FA_ERR_INVALID_ARG"]
+    assert fa.lib.fa_bwd(*args, 1, 1, 0, 64, F(0.125), 0, None, 0, None) == C["FA_OK"]
+
+
+def test_noalloc_limit_is_checked_first():
+    limit = fa.lib.fa_bwd_noalloc_max_bytes()
+    assert limit == 64 << 20
+    assert fa.fa_bwd_workspace_size(1, 32, 4096, 128) > limit
+    st = fa.lib.fa_bwd_noalloc(*([4096] * 9), 1, 32, 4096, 128, F(0.1), 0, None)
+    assert st == C["FA_ERR_SCRATCH_LIMIT"]
+    assert fa.lib.fa_bwd_noalloc(*([4096] * 9), 1, 1, 16, 96, F(0.1), 0, None) == C["FA_ERR_UNSUPPORTED"]
