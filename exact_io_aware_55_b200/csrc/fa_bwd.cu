@@ -46,10 +46,10 @@ constexpr int kTile = 128;
 constexpr int kThreads = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 // Registers per thread after re-balancing.  Launch: 512 threads x 128 = 65536;
-// after: warpgroup 0 (producer, MMA, 2 idle warps) 80, the two P/dS
-// warpgroups 144, the dQ warpgroup 144: 128 x (80 + 2 x 144 + 144) = 65536.
-constexpr uint32_t kRegsWG0 = 80;
-constexpr uint32_t kRegsPdS = 144;
+// after: warpgroup 0 (producer, MMA, 2 idle warps) 96, the two P/dS
+// warpgroups 136, the dQ warpgroup 144: 128 x (96 + 2 x 136 + 144) = 65536.
+constexpr uint32_t kRegsWG0 = 96;
+constexpr uint32_t kRegsPdS = 136;
 constexpr uint32_t kRegsDQ = 144;
 static_assert(128 * (kRegsWG0 + 2 * kRegsPdS + kRegsDQ) <= 512 * 128, "register split exceeds the launch allocation");
 
@@ -220,103 +220,112 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsWG0>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmdO);
-      const uint64_t pol_q = policy_evict_last();    // Q/dO tiles are re-read by every key tile
-      const uint64_t pol_kv = policy_evict_first();  // K/V tiles are read once
-      mbar_arrive_expect_tx(&bars->kv_full, 2 * S::kTileBytes);
+    // The whole warp runs this loop; elect.sync picks the lane that issues.
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmdO);
+    const uint64_t pol_q = policy_evict_last();    // Q/dO tiles are re-read by every key tile
+    const uint64_t pol_kv = policy_evict_first();  // K/V tiles are read once
+    mbar_arrive_expect_tx_e(&bars->kv_full, 2 * S::kTileBytes);
+#pragma unroll
+    for (int c = 0; c < S::kChunks; ++c) {
+      tma_load_3d_hint_e(sK + c * 16384, &tmK, &bars->kv_full, c * 64, j * kTile, bh, pol_kv);
+      tma_load_3d_hint_e(sV + c * 16384, &tmV, &bars->kv_full, c * 64, j * kTile, bh, pol_kv);
+    }
+    for (int it = 0; it < n_iter; ++it) {
+      const int s = it % NST;
+      const int i = i_begin + it;
+      if (it >= NST) {
+        if (!mbar_wait_warp(&bars->qdo_empty[s], ((it / NST) + 1) & 1, wc, WAIT_BWD_QDO_EMPTY)) break;
+      }
+      mbar_arrive_expect_tx_e(&bars->qdo_full[s], 2 * S::kTileBytes + 1024);
+#pragma unroll
       for (int c = 0; c < S::kChunks; ++c) {
-        tma_load_3d_hint(sK + c * 16384, &tmK, &bars->kv_full, c * 64, j * kTile, bh, pol_kv);
-        tma_load_3d_hint(sV + c * 16384, &tmV, &bars->kv_full, c * 64, j * kTile, bh, pol_kv);
-      }
-      for (int it = 0; it < n_iter; ++it) {
-        const int s = it % NST;
-        const int i = i_begin + it;
-        if (it >= NST) {
-          if (!mbar_wait(&bars->qdo_empty[s], ((it / NST) + 1) & 1, wc, WAIT_BWD_QDO_EMPTY)) break;
-        }
-        mbar_arrive_expect_tx(&bars->qdo_full[s], 2 * S::kTileBytes + 1024);
-        for (int c = 0; c < S::kChunks; ++c) {
-          tma_load_3d_hint(sQ + s * S::kTileBytes + c * 16384, &tmQ, &bars->qdo_full[s], c * 64, i * kTile, bh,
+        tma_load_3d_hint_e(sQ + s * S::kTileBytes + c * 16384, &tmQ, &bars->qdo_full[s], c * 64, i * kTile, bh,
                            pol_q);
-          tma_load_3d_hint(sdO + s * S::kTileBytes + c * 16384, &tmdO, &bars->qdo_full[s], c * 64, i * kTile,
-                           bh, pol_q);
-        }
-        const size_t srow = size_t(bh) * args.Np + size_t(i) * kTile;
-        bulk_load(sStat + s * 256, args.neg_lse2 + srow, 512, &bars->qdo_full[s]);
-        bulk_load(sStat + s * 256 + 128, args.neg_dvec + srow, 512, &bars->qdo_full[s]);
+        tma_load_3d_hint_e(sdO + s * S::kTileBytes + c * 16384, &tmdO, &bars->qdo_full[s], c * 64, i * kTile, bh,
+                           pol_q);
       }
+      const size_t srow = size_t(bh) * args.Np + size_t(i) * kTile;
+      bulk_load_e(sStat + s * 256, args.neg_lse2 + srow, 512, &bars->qdo_full[s]);
+      bulk_load_e(sStat + s * 256 + 128, args.neg_dvec + srow, 512, &bars->qdo_full[s]);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
-      const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sdOa = smem_u32(sdO),
-                     sdSa = smem_u32(sdS);
-      const uint32_t tR1 = tmem + S::kColR1, tR2 = tmem + S::kColR2;
-      // X^T tile = A_tile B_tile^T over d, both K-major (S^T = K Q^T, dP^T = V dO^T).
-      auto issue_xt = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
+    // Warp-uniform: every lane walks the loop and waits; one elected lane
+    // issues each tcgen05 instruction and every commit.  Descriptors: a base
+    // per operand, then constant byte offsets (>> 4).
+    const uint32_t tR1 = tmem + S::kColR1, tR2 = tmem + S::kColR2;
+    const uint64_t dK_k = sdesc_sw128(smem_u32(sK), 16, 1024);      // K tile, K-major (A of S^T)
+    const uint64_t dV_k = sdesc_sw128(smem_u32(sV), 16, 1024);      // V tile, K-major (A of dP^T)
+    const uint64_t dQ_k = sdesc_sw128(smem_u32(sQ), 16, 1024);      // Q stages, K-major (B of S^T)
+    const uint64_t ddO_k = sdesc_sw128(smem_u32(sdO), 16, 1024);    // dO stages, K-major (B of dP^T)
+    const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), 16384, 1024);  // Q stages, MN-major (B of dK)
+    const uint64_t ddO_mn = sdesc_sw128(smem_u32(sdO), 16384, 1024);// dO stages, MN-major (B of dV)
+    const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), 16384, 1024);  // K tile, MN-major (A of dQ^T)
+    const uint64_t ddS_k = sdesc_sw128(smem_u32(sdS), 16, 1024);    // dS^T, K-major (A of dK)
+    const uint64_t ddS_mn = sdesc_sw128(smem_u32(sdS), 16384, 1024);// dS^T, MN-major (B of dQ^T)
+    constexpr uint64_t kTileD = uint64_t(S::kTileBytes >> 4);
+    // X^T tile = A_tile B_tile^T over d, both K-major (S^T = K Q^T, dP^T = V dO^T).
+    auto issue_xt = [&](uint32_t d_tmem, uint64_t a, uint64_t b) {
 #pragma unroll
-        for (int ks = 0; ks < S::kKSteps; ++ks) {
-          const uint32_t off = uint32_t((ks >> 2) * 16384 + (ks & 3) * 32);
-          mma_f16_ss(d_tmem, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024), S::kIdSS,
-                     ks > 0);
-        }
-      };
-      bool ok = mbar_wait(&bars->kv_full, 0, wc, WAIT_BWD_KV) && mbar_wait(&bars->qdo_full[0], 0, wc, WAIT_BWD_QDO);
-      if (ok) {
-        tc_fence_after();
-        issue_xt(tR1, sKa, sQa);                       // S^T_0
-        tc_commit(&bars->s_ready);
-        for (int it = 0; it < n_iter; ++it) {
-          const int s = it % NST;
-          const uint32_t qa = sQa + s * S::kTileBytes, doa = sdOa + s * S::kTileBytes;
-          if (it > 0) {
-            if (!mbar_wait(&bars->dq_free, (it - 1) & 1, wc, WAIT_BWD_DQ_FREE)) { ok = false; break; }
-            tc_fence_after();
-          }
-          issue_xt(tR2, sVa, doa);                     // dP^T_it
-          tc_commit(&bars->dp_ready);
-          if (!mbar_wait(&bars->p_ready, it & 1, wc, WAIT_BWD_P)) { ok = false; break; }
-          tc_fence_after();
-          // dV += P^T dO: A = P^T (TMEM R1, bf16), B = dO MN-major; 16 queries per step.
-#pragma unroll
-          // P^T of queries 0-63 sits in R1 columns [0,32), of queries 64-127 in [96,128).
-          for (int kt = 0; kt < 8; ++kt)
-            mma_f16_ts(tmem + S::kColDV, tR1 + kt * 8 + (kt >= 4 ? 64 : 0), sdesc_sw128(doa + kt * 2048, 16384, 1024),
-                       S::kIdKmaj, (it > 0 || kt > 0) ? 1u : 0u);
-          if (it + 1 < n_iter) {                        // S^T of the next query tile
-            const int sn = (it + 1) % NST;
-            if (!mbar_wait(&bars->qdo_full[sn], ((it + 1) / NST) & 1, wc, WAIT_BWD_QDO)) { ok = false; break; }
-            tc_fence_after();
-            issue_xt(tR1, sKa, sQa + sn * S::kTileBytes);
-            tc_commit(&bars->s_ready);
-          }
-          if (!mbar_wait(&bars->ds_ready, it & 1, wc, WAIT_BWD_DS)) { ok = false; break; }
-          tc_fence_after();
-          // dK += dS^T Q: A = dS^T K-major (rows = keys, 128 queries), B = Q MN-major.
-#pragma unroll
-          for (int kt = 0; kt < 8; ++kt) {
-            const uint32_t off = uint32_t((kt >> 2) * 16384 + (kt & 3) * 32);
-            mma_f16_ss(tmem + S::kColDK, sdesc_sw128(sdSa + off, 16, 1024),
-                       sdesc_sw128(qa + kt * 2048, 16384, 1024), S::kIdKmaj, (it > 0 || kt > 0) ? 1u : 0u);
-          }
-          // dQ^T = K^T dS^T: A = K read MN-major (M = d), B = the dS^T bytes read
-          // MN-major (N = queries); 16 keys per step.  The transposed product puts
-          // d on the TMEM lanes, so each dQ row update is one coalesced line.
-#pragma unroll
-          for (int kt = 0; kt < 8; ++kt)
-            mma_f16_ss(tR2, sdesc_sw128(sKa + kt * 2048, 16384, 1024), sdesc_sw128(sdSa + kt * 2048, 16384, 1024),
-                       S::kIdDQT, kt > 0 ? 1u : 0u);
-          tc_commit(&bars->dq_ready);
-          tc_commit(&bars->ds_free);
-          tc_commit(&bars->qdo_empty[s]);
-        }
-        tc_commit(&bars->final_);
-        if (ok) (void)mbar_wait(&bars->final_, 0, wc, WAIT_BWD_FINAL);
+      for (int ks = 0; ks < S::kKSteps; ++ks) {
+        const uint64_t off = uint64_t(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+        mma_f16_ss_e(d_tmem, a + off, b + off, S::kIdSS, ks > 0 ? 1u : 0u);
       }
+    };
+    bool ok = mbar_wait_warp(&bars->kv_full, 0, wc, WAIT_BWD_KV) &&
+              mbar_wait_warp(&bars->qdo_full[0], 0, wc, WAIT_BWD_QDO);
+    if (ok) {
+      tc_fence_after();
+      issue_xt(tR1, dK_k, dQ_k);                       // S^T_0
+      tc_commit_e(&bars->s_ready);
+      for (int it = 0; it < n_iter; ++it) {
+        const int s = it % NST;
+        const uint64_t st = uint64_t(s) * kTileD;
+        if (it > 0) {
+          if (!mbar_wait_warp(&bars->dq_free, (it - 1) & 1, wc, WAIT_BWD_DQ_FREE)) { ok = false; break; }
+          tc_fence_after();
+        }
+        issue_xt(tR2, dV_k, ddO_k + st);               // dP^T_it
+        tc_commit_e(&bars->dp_ready);
+        if (!mbar_wait_warp(&bars->p_ready, it & 1, wc, WAIT_BWD_P)) { ok = false; break; }
+        tc_fence_after();
+        // dV += P^T dO: A = P^T (TMEM R1, bf16), B = dO MN-major; 16 queries per step.
+        // P^T of queries 0-63 sits in R1 columns [0,32), of queries 64-127 in [96,128).
+#pragma unroll
+        for (int kt = 0; kt < 8; ++kt)
+          mma_f16_ts_e(tmem + S::kColDV, tR1 + kt * 8 + (kt >= 4 ? 64 : 0), ddO_mn + st + uint64_t(kt * 128),
+                       S::kIdKmaj, (it > 0 || kt > 0) ? 1u : 0u);
+        if (it + 1 < n_iter) {                        // S^T of the next query tile
+          const int sn = (it + 1) % NST;
+          if (!mbar_wait_warp(&bars->qdo_full[sn], ((it + 1) / NST) & 1, wc, WAIT_BWD_QDO)) { ok = false; break; }
+          tc_fence_after();
+          issue_xt(tR1, dK_k, dQ_k + uint64_t(sn) * kTileD);
+          tc_commit_e(&bars->s_ready);
+        }
+        if (!mbar_wait_warp(&bars->ds_ready, it & 1, wc, WAIT_BWD_DS)) { ok = false; break; }
+        tc_fence_after();
+        // dK += dS^T Q: A = dS^T K-major (rows = keys, 128 queries), B = Q MN-major.
+#pragma unroll
+        for (int kt = 0; kt < 8; ++kt) {
+          const uint64_t off = uint64_t(((kt >> 2) * 16384 + (kt & 3) * 32) >> 4);
+          mma_f16_ss_e(tmem + S::kColDK, ddS_k + off, dQ_mn + st + uint64_t(kt * 128), S::kIdKmaj,
+                       (it > 0 || kt > 0) ? 1u : 0u);
+        }
+        // dQ^T = K^T dS^T: A = K read MN-major (M = d), B = the dS^T bytes read
+        // MN-major (N = queries); 16 keys per step.  The transposed product puts
+        // d on the TMEM lanes, so each dQ row update is one coalesced line.
+#pragma unroll
+        for (int kt = 0; kt < 8; ++kt)
+          mma_f16_ss_e(tR2, dK_mn + uint64_t(kt * 128), ddS_mn + uint64_t(kt * 128), S::kIdDQT, kt > 0 ? 1u : 0u);
+        tc_commit_e(&bars->dq_ready);
+        tc_commit_e(&bars->ds_free);
+        tc_commit_e(&bars->qdo_empty[s]);
+      }
+      tc_commit_e(&bars->final_);
+      if (ok) (void)mbar_wait_warp(&bars->final_, 0, wc, WAIT_BWD_FINAL);
     }
   }
   } else if (warp < 12) {

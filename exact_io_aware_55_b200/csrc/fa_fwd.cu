@@ -40,9 +40,9 @@ constexpr int kThreads = 384;   // 12 warps
 constexpr float kRescaleThresh = 8.0f;
 // Registers per thread after re-balancing: warpgroup 0 (producer, MMA, two
 // idle warps) gives registers to the two softmax warpgroups.  Launch: 384
-// threads x 168 = 64512; after: 128 x 64 + 256 x 216 = 63488.
-constexpr uint32_t kRegsWG0 = 64;
-constexpr uint32_t kRegsSoftmax = 216;
+// threads x 168 = 64512; after: 128 x 80 + 256 x 208 = 63488.
+constexpr uint32_t kRegsWG0 = 80;
+constexpr uint32_t kRegsSoftmax = 208;
 static_assert(128 * kRegsWG0 + 256 * kRegsSoftmax <= 384 * 168, "register split exceeds the launch allocation");
 constexpr float kLn2 = 0.69314718055994530942f;
 
@@ -194,109 +194,118 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsWG0>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      const uint64_t pol_kv = policy_evict_last();
-      const uint64_t pol_q = policy_evict_first();
-      int nq = 0;
-      for (int g = 0; g < kNQT; ++g) nq += (T[g] > 0);
-      mbar_arrive_expect_tx(&bars->q, nq * S::kTileBytes);
-      for (int g = 0; g < kNQT; ++g) {
-        if (T[g] == 0) continue;
-        for (int c = 0; c < S::kChunks; ++c)
-          tma_load_3d_hint(sQ + g * S::kTileBytes + c * 16384, &tmQ, &bars->q, c * S::kChunkElems, q0[g], bh,
+    // The whole warp runs this loop; elect.sync picks the lane that issues.
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    const uint64_t pol_kv = policy_evict_last();
+    const uint64_t pol_q = policy_evict_first();
+    int nq = 0;
+#pragma unroll
+    for (int g = 0; g < kNQT; ++g) nq += (T[g] > 0);
+    mbar_arrive_expect_tx_e(&bars->q, nq * S::kTileBytes);
+#pragma unroll
+    for (int g = 0; g < kNQT; ++g) {
+      if (T[g] == 0) continue;
+#pragma unroll
+      for (int c = 0; c < S::kChunks; ++c)
+        tma_load_3d_hint_e(sQ + g * S::kTileBytes + c * 16384, &tmQ, &bars->q, c * S::kChunkElems, q0[g], bh,
                            pol_q);
+    }
+    for (int j = 0; j < Tmax; ++j) {
+      const int s = j % NST;
+      if (j >= NST) {
+        if (!mbar_wait_warp(&bars->kv_empty[s], ((j / NST) + 1) & 1, wc, WAIT_FWD_KV_EMPTY)) break;
       }
-      for (int j = 0; j < Tmax; ++j) {
-        const int s = j % NST;
-        if (j >= NST) {
-          if (!mbar_wait(&bars->kv_empty[s], ((j / NST) + 1) & 1, wc, WAIT_FWD_KV_EMPTY)) break;
-        }
-        mbar_arrive_expect_tx(&bars->k_full[s], S::kTileBytes);
-        for (int c = 0; c < S::kChunks; ++c)
-          tma_load_3d_hint(sK + s * S::kTileBytes + c * 16384, &tmK, &bars->k_full[s], c * S::kChunkElems,
+      mbar_arrive_expect_tx_e(&bars->k_full[s], S::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < S::kChunks; ++c)
+        tma_load_3d_hint_e(sK + s * S::kTileBytes + c * 16384, &tmK, &bars->k_full[s], c * S::kChunkElems,
                            j * kBN, bh, pol_kv);
-        mbar_arrive_expect_tx(&bars->v_full[s], S::kTileBytes);
-        for (int c = 0; c < S::kChunks; ++c)
-          tma_load_3d_hint(sV + s * S::kTileBytes + c * 16384, &tmV, &bars->v_full[s], c * S::kChunkElems,
+      mbar_arrive_expect_tx_e(&bars->v_full[s], S::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < S::kChunks; ++c)
+        tma_load_3d_hint_e(sV + s * S::kTileBytes + c * 16384, &tmV, &bars->v_full[s], c * S::kChunkElems,
                            j * kBN, bh, pol_kv);
-      }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      auto issue_s = [&](int g, int s) {
-        const uint32_t d_tmem = tmem + uint32_t(g * 128);
+    // Warp-uniform: every lane walks the loop and waits; one elected lane
+    // issues each tcgen05 instruction (and all commits, so they track its MMAs).
+    // Descriptors: a base per operand, then constant byte offsets (>> 4).
+    const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);       // K-major
+    const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);       // K-major
+    const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16384, 1024);    // MN-major
+    constexpr uint64_t kTileD = uint64_t(S::kTileBytes >> 4);
+    auto issue_s = [&](int g, int s) {
+      const uint32_t d_tmem = tmem + uint32_t(g * 128);
+      const uint64_t a = dQ0 + uint64_t(g) * kTileD, b = dK0 + uint64_t(s) * kTileD;
 #pragma unroll
-        for (int ks = 0; ks < S::kSSteps; ++ks) {
-          const uint32_t off = uint32_t((ks >> 2) * 16384 + (ks & 3) * 32);
-          const uint64_t a = sdesc_sw128(sQa + g * S::kTileBytes + off, 16, 1024);
-          const uint64_t b = sdesc_sw128(sKa + s * S::kTileBytes + off, 16, 1024);
-          if constexpr (FP8)
-            mma_f8_ss(d_tmem, a, b, S::kIdS, ks > 0);
-          else
-            mma_f16_ss(d_tmem, a, b, S::kIdS, ks > 0);
-        }
-      };
-      auto issue_pv = [&](int g, int s, bool acc) {
-        const uint32_t d_tmem = tmem + uint32_t(kNQT * 128 + g * D);
-        const uint32_t p_tmem = tmem + uint32_t(g * 128);
-#pragma unroll
-        for (int kt = 0; kt < S::kPVSteps; ++kt) {
-          const uint64_t b = sdesc_sw128(sVa + s * S::kTileBytes + kt * S::kPVRows * 128, 16384, 1024);
-          if constexpr (FP8)
-            mma_f8_ts(d_tmem, p_tmem + kt * 8, b, S::kIdPV, (acc || kt > 0) ? 1u : 0u);
-          else
-            mma_f16_ts(d_tmem, p_tmem + kt * 8, b, S::kIdPV, (acc || kt > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(&bars->q, 0, wc, WAIT_FWD_Q) &&
-                mbar_wait(&bars->k_full[0], 0, wc, WAIT_FWD_K);
-      if (ok) {
-        tc_fence_after();
-        for (int g = 0; g < kNQT; ++g) {
-          if (T[g] == 0) continue;
-          issue_s(g, 0);
-          tc_commit(&bars->s_full[g]);
-        }
-        for (int j = 0; j < Tmax && ok; ++j) {
-          const int s = j % NST;
-          if (!mbar_wait(&bars->v_full[s], (j / NST) & 1, wc, WAIT_FWD_V)) break;
-          tc_fence_after();
-          bool k_next_ready = false;
-          for (int g = 0; g < kNQT; ++g) {
-            if (j >= T[g]) continue;
-            if (!mbar_wait(&bars->p_full[g], j & 1, wc, WAIT_FWD_P)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_pv(g, s, j > 0);
-            if (j + 1 < T[g]) {
-              if (!k_next_ready) {
-                const int sn = (j + 1) % NST;
-                if (!mbar_wait(&bars->k_full[sn], ((j + 1) / NST) & 1, wc, WAIT_FWD_K)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
-                k_next_ready = true;
-              }
-              issue_s(g, (j + 1) % NST);
-              tc_commit(&bars->s_full[g]);
-            } else {
-              tc_commit(&bars->o_final[g]);
-            }
-          }
-          tc_commit(&bars->kv_empty[s]);
-        }
-        // Let the last commit land before the CTA can exit.
-        if (ok && Tmax > 0)
-          (void)mbar_wait(&bars->kv_empty[(Tmax - 1) % NST], ((Tmax - 1) / NST) & 1, wc, WAIT_FWD_KV_EMPTY);
+      for (int ks = 0; ks < S::kSSteps; ++ks) {
+        const uint64_t off = uint64_t(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+        if constexpr (FP8)
+          mma_f8_ss_e(d_tmem, a + off, b + off, S::kIdS, ks > 0 ? 1u : 0u);
+        else
+          mma_f16_ss_e(d_tmem, a + off, b + off, S::kIdS, ks > 0 ? 1u : 0u);
       }
+    };
+    auto issue_pv = [&](int g, int s, bool acc) {
+      const uint32_t d_tmem = tmem + uint32_t(kNQT * 128 + g * D);
+      const uint32_t p_tmem = tmem + uint32_t(g * 128);
+      const uint64_t b = dV0 + uint64_t(s) * kTileD;
+#pragma unroll
+      for (int kt = 0; kt < S::kPVSteps; ++kt) {
+        const uint64_t off = uint64_t((kt * S::kPVRows * 128) >> 4);
+        if constexpr (FP8)
+          mma_f8_ts_e(d_tmem, p_tmem + kt * 8, b + off, S::kIdPV, (acc || kt > 0) ? 1u : 0u);
+        else
+          mma_f16_ts_e(d_tmem, p_tmem + kt * 8, b + off, S::kIdPV, (acc || kt > 0) ? 1u : 0u);
+      }
+    };
+    bool ok = mbar_wait_warp(&bars->q, 0, wc, WAIT_FWD_Q) && mbar_wait_warp(&bars->k_full[0], 0, wc, WAIT_FWD_K);
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int g = 0; g < kNQT; ++g) {
+        if (T[g] == 0) continue;
+        issue_s(g, 0);
+        tc_commit_e(&bars->s_full[g]);
+      }
+      for (int j = 0; j < Tmax && ok; ++j) {
+        const int s = j % NST;
+        if (!mbar_wait_warp(&bars->v_full[s], (j / NST) & 1, wc, WAIT_FWD_V)) break;
+        tc_fence_after();
+        bool k_next_ready = false;
+#pragma unroll
+        for (int g = 0; g < kNQT; ++g) {
+          if (j >= T[g] || !ok) continue;
+          if (!mbar_wait_warp(&bars->p_full[g], j & 1, wc, WAIT_FWD_P)) {
+            ok = false;
+            continue;
+          }
+          tc_fence_after();
+          issue_pv(g, s, j > 0);
+          if (j + 1 < T[g]) {
+            if (!k_next_ready) {
+              const int sn = (j + 1) % NST;
+              if (!mbar_wait_warp(&bars->k_full[sn], ((j + 1) / NST) & 1, wc, WAIT_FWD_K)) {
+                ok = false;
+                continue;
+              }
+              tc_fence_after();
+              k_next_ready = true;
+            }
+            issue_s(g, (j + 1) % NST);
+            tc_commit_e(&bars->s_full[g]);
+          } else {
+            tc_commit_e(&bars->o_final[g]);
+          }
+        }
+        tc_commit_e(&bars->kv_empty[s]);
+      }
+      // Let the last commit land before the CTA can exit.
+      if (ok && Tmax > 0)
+        (void)mbar_wait_warp(&bars->kv_empty[(Tmax - 1) % NST], ((Tmax - 1) / NST) & 1, wc, WAIT_FWD_KV_EMPTY);
     }
   }
   } else {

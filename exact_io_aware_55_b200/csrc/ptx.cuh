@@ -218,6 +218,66 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// ---------------------------------------------- elected-lane issue forms
+// Called by every lane of a converged warp; elect.sync picks one lane (the
+// lowest) to execute the instruction.  Keeping the issuing code warp-uniform
+// lets the compiler hold descriptors in uniform registers: tcgen05.mma issued
+// this way streams at the tensor-pipe rate, whereas issuing from a one-lane
+// divergent branch costs a multiple of that per instruction.
+#define FA_MMA_ELECT(kind, aop, aconstraint)                                                            \
+  asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"       \
+               "@e tcgen05.mma.cta_group::1.kind::" kind " [%0], " aop ", %2, %3, p;\n\t}" ::"r"(d_tmem),  \
+               aconstraint(a), "l"(b_desc), "r"(idesc), "r"(accumulate)                                 \
+               : "memory")
+__device__ __forceinline__ void mma_f16_ss_e(uint32_t d_tmem, uint64_t a, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  FA_MMA_ELECT("f16", "%1", "l");
+}
+__device__ __forceinline__ void mma_f16_ts_e(uint32_t d_tmem, uint32_t a, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  FA_MMA_ELECT("f16", "[%1]", "r");
+}
+__device__ __forceinline__ void mma_f8_ss_e(uint32_t d_tmem, uint64_t a, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  FA_MMA_ELECT("f8f6f4", "%1", "l");
+}
+__device__ __forceinline__ void mma_f8_ts_e(uint32_t d_tmem, uint32_t a, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  FA_MMA_ELECT("f8f6f4", "[%1]", "r");
+}
+#undef FA_MMA_ELECT
+__device__ __forceinline__ void tc_commit_e(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_e(uint64_t* bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+      "r"(bytes)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_hint_e(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                                   int c2, uint64_t policy) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;\n\t}" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load_e(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100
 // descriptor version 1.  `saddr` is the shared-window byte address of the
 // operand's first element; lbo/sbo are byte strides (leading / stride
