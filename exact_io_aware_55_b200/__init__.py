@@ -15,7 +15,8 @@ import torch
 from ._lib import FA_OK, FAError, LIB_PATH, STATUS_CODES, STATUS_NAMES, check, lib, strerror
 
 __all__ = [
-    "FAError", "LIB_PATH", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_size", "fa_device_status",
+    "FAError", "LIB_PATH", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size",
+    "fa_device_status",
     "fa_watchdog_selftest", "attention_forward", "attention_backward", "attention_forward_fp8", "lib",
     "STATUS_NAMES", "STATUS_CODES", "strerror",
 ]
@@ -85,6 +86,18 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, workspac
                      B, H, N, d, float(scale), int(bool(causal)), _ptr(workspace), wbytes, _stream_ptr(stream)))
 
 
+def fa_bwd_deterministic(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, workspace,
+                         stream=None) -> None:
+    """As fa_bwd, with dQ from a separate atomic-free pass: bit-reproducible results."""
+    B, H, N, d = _shape(q)
+    _check_tensors((B, H, N, d), torch.bfloat16, q, k, v, o, do, dq, dk, dv)
+    _check_tensors((B, H, N), torch.float32, lse)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.fa_bwd_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), B, H, N, d, float(scale), int(bool(causal)), _ptr(workspace), wbytes,
+                                   _stream_ptr(stream)))
+
+
 def fa_device_status(stream=None):
     """(status, where) of the device status word; synchronises the stream and clears it."""
     where = ctypes.c_uint32(0)
@@ -120,12 +133,13 @@ def attention_forward_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale: fl
 
 
 def attention_backward(q, k, v, o, do, lse, scale: float | None = None, causal: bool = False, workspace=None,
-                       stream=None):
-    """Allocates dQ, dK, dV (and the workspace unless given) with torch and runs fa_bwd."""
+                       stream=None, deterministic: bool = False):
+    """Allocates dQ, dK, dV (and the workspace unless given) with torch and runs
+    fa_bwd (or fa_bwd_deterministic)."""
     B, H, N, d = _shape(q)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
         workspace = torch.empty(max(1, fa_bwd_workspace_size(B, H, N, d)), dtype=torch.uint8, device=q.device)
-    fa_bwd(q, k, v, o, do, lse, dq, dk, dv, _default_scale(d) if scale is None else scale, causal, workspace,
-           stream)
+    fn = fa_bwd_deterministic if deterministic else fa_bwd
+    fn(q, k, v, o, do, lse, dq, dk, dv, _default_scale(d) if scale is None else scale, causal, workspace, stream)
     return dq, dk, dv

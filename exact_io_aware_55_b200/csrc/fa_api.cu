@@ -186,9 +186,32 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return ws_layout(static_cast<long long>(B) * H, N, d).total;
 }
 
+namespace {
+fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                     void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                     void* workspace, size_t workspace_bytes, void* stream, bool deterministic);
+}  // namespace
+
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                  void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_common(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes, stream,
+                    false);
+}
+
+fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                               const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                               float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_common(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes, stream,
+                    true);
+}
+
+}  // extern "C"
+
+namespace {
+fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                     void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                     void* workspace, size_t workspace_bytes, void* stream, bool deterministic) {
   bool empty = false;
   fa_status st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK) return st;
@@ -223,8 +246,12 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.BH = BH;
   a.c_log2 = scale * kLog2e;
   a.scale = scale;
-  return launch_status(fa::launch_bwd(tq, tk, tv, tdo, a, d, causal != 0, static_cast<cudaStream_t>(stream)));
+  return launch_status(
+      fa::launch_bwd(tq, tk, tv, tdo, a, d, causal != 0, deterministic, static_cast<cudaStream_t>(stream)));
 }
+}  // namespace
+
+extern "C" {
 
 const char* fa_strerror(fa_status s) {
   switch (s) {

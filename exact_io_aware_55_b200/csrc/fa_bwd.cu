@@ -152,7 +152,10 @@ __device__ __forceinline__ void red_add_f32(float* addr, float a) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-template <int D, bool CAUSAL>
+// DQ = false: deterministic mode; this kernel produces dK and dV only and
+// the dQ^T product, its reductions and the dQ warpgroup are skipped (dQ comes
+// from bwd_dq_kernel).
+template <int D, bool CAUSAL, bool DQ>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -284,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < n_iter; ++it) {
         const int s = it % NST;
         const uint64_t st = uint64_t(s) * kTileD;
-        if (it > 0) {
+        if (DQ && it > 0) {
           if (!mbar_wait_warp(&bars->dq_free, (it - 1) & 1, wc, WAIT_BWD_DQ_FREE)) { ok = false; break; }
           tc_fence_after();
         }
@@ -317,10 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dQ^T = K^T dS^T: A = K read MN-major (M = d), B = the dS^T bytes read
         // MN-major (N = queries); 16 keys per step.  The transposed product puts
         // d on the TMEM lanes, so each dQ row update is one coalesced line.
+        if constexpr (DQ) {
 #pragma unroll
-        for (int kt = 0; kt < 8; ++kt)
-          mma_f16_ss_e(tR2, dK_mn + uint64_t(kt * 128), ddS_mn + uint64_t(kt * 128), S::kIdDQT, kt > 0 ? 1u : 0u);
-        tc_commit_e(&bars->dq_ready);
+          for (int kt = 0; kt < 8; ++kt)
+            mma_f16_ss_e(tR2, dK_mn + uint64_t(kt * 128), ddS_mn + uint64_t(kt * 128), S::kIdDQT, kt > 0 ? 1u : 0u);
+          tc_commit_e(&bars->dq_ready);
+        }
         tc_commit_e(&bars->ds_free);
         tc_commit_e(&bars->qdo_empty[s]);
       }
@@ -440,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else {
+  } else if (DQ) {
     regs_inc<kRegsDQ>();
     // ---------------------------------------------------------- dQ group
     // dQ^T tile in TMEM R2: lane = d index, column = query.  With M = d = 128
@@ -480,27 +485,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DQ>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
   // 1) preprocess + zero the dQ accumulator
   constexpr int RPB = 256 / (D / 8);
   const long long rows = (long long)a.BH * a.Np;
   const int row_blocks = int((rows + RPB - 1) / RPB);
-  const long long dq_vec4 = (long long)a.BH * a.N * D / 4;
-  const int zero_blocks = int(std::min<long long>((dq_vec4 + 255) / 256, 148LL * 8));
+  const long long dq_vec4 = DQ ? (long long)a.BH * a.N * D / 4 : 0;
+  const int zero_blocks = DQ ? int(std::min<long long>((dq_vec4 + 255) / 256, 148LL * 8)) : 0;
   bwd_pre_kernel<D><<<row_blocks + zero_blocks, 256, 0, stream>>>(a, row_blocks, dq_vec4);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // 2) main kernel
   constexpr size_t smem = bwd_smem_bytes<D>();
-  auto kern = bwd_kernel<D, CAUSAL>;
+  auto kern = bwd_kernel<D, CAUSAL, DQ>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((a.N + kTile - 1) / kTile, a.BH);
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if constexpr (!DQ) {
+    // 3) deterministic dQ: query-tile-stationary pass, written once as bf16
+    return launch_bwd_dq<D, CAUSAL>(tq, tk, tv, tdo, a, stream);
+  }
   // 3) dQ -> bf16
   const long long n8 = (long long)a.BH * a.N * D / 8;
   const int fin_blocks = int(std::min<long long>((n8 + 255) / 256, 148LL * 8));
@@ -511,11 +520,17 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 }  // namespace
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const BwdArgs& a, int d, bool causal, cudaStream_t stream) {
-  if (d == 64) return causal ? launch_bwd_t<64, true>(tq, tk, tv, tdo, a, stream)
-                             : launch_bwd_t<64, false>(tq, tk, tv, tdo, a, stream);
-  return causal ? launch_bwd_t<128, true>(tq, tk, tv, tdo, a, stream)
-                : launch_bwd_t<128, false>(tq, tk, tv, tdo, a, stream);
+                       const BwdArgs& a, int d, bool causal, bool deterministic, cudaStream_t stream) {
+  if (deterministic) {
+    if (d == 64) return causal ? launch_bwd_t<64, true, false>(tq, tk, tv, tdo, a, stream)
+                               : launch_bwd_t<64, false, false>(tq, tk, tv, tdo, a, stream);
+    return causal ? launch_bwd_t<128, true, false>(tq, tk, tv, tdo, a, stream)
+                  : launch_bwd_t<128, false, false>(tq, tk, tv, tdo, a, stream);
+  }
+  if (d == 64) return causal ? launch_bwd_t<64, true, true>(tq, tk, tv, tdo, a, stream)
+                             : launch_bwd_t<64, false, true>(tq, tk, tv, tdo, a, stream);
+  return causal ? launch_bwd_t<128, true, true>(tq, tk, tv, tdo, a, stream)
+                : launch_bwd_t<128, false, true>(tq, tk, tv, tdo, a, stream);
 }
 
 }  // namespace fa

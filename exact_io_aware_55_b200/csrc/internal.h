@@ -27,6 +27,17 @@ enum WaitSite : uint32_t {
   WAIT_BWD_DQ = 24,
   WAIT_BWD_DQ_FREE = 25,
   WAIT_BWD_FINAL = 26,
+  WAIT_DQ_QDO = 32,
+  WAIT_DQ_K = 33,
+  WAIT_DQ_V = 34,
+  WAIT_DQ_KV_EMPTY = 35,
+  WAIT_DQ_S = 36,
+  WAIT_DQ_DP = 37,
+  WAIT_DQ_SFREE = 38,
+  WAIT_DQ_DPFREE = 39,
+  WAIT_DQ_DS = 40,
+  WAIT_DQ_DSFREE = 41,
+  WAIT_DQ_FINAL = 42,
   WAIT_SELFTEST = 99,
 };
 
@@ -65,7 +76,13 @@ cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const 
 cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdArgs& a, int d, bool causal, cudaStream_t stream);
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdArgs& a, int d, bool causal, cudaStream_t stream);
+                       const CUtensorMap& tdo, const BwdArgs& a, int d, bool causal, bool deterministic,
+                       cudaStream_t stream);
+// Deterministic dQ pass (one 128-query tile per CTA, no atomics); defined in
+// fa_bwd_dq.cu, launched by launch_bwd after the dK/dV kernel.
+template <int D, bool CAUSAL>
+cudaError_t launch_bwd_dq(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_watchdog_selftest(uint64_t limit_ns, cudaStream_t stream);
 
 }  // namespace fa

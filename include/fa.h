@@ -109,6 +109,19 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward pass with a deterministic dQ: same arguments, outputs and workspace
+ * as fa_bwd, but dQ is produced by a separate query-tile-parallel pass that
+ * recomputes S, P and dP per query tile and accumulates dQ_i += dS K_j in
+ * on-chip memory, writing each row once (no atomics).  Repeated calls on the
+ * same inputs return bit-identical dQ, dK and dV.  Costs two more GEMMs per
+ * tile pair (the recomputed S and dP) than fa_bwd.
+ */
+FA_API fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                      const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                                      float scale, int causal, void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
+/*
  * Forward pass with float8 e4m3 inputs and per-tensor scales ("What changed
  * between FlashAttention 1, 2, and 3?": low-precision FP8 forward).
  * The real inputs are q8 * q_descale, k8 * k_descale, v8 * v_descale.  The
