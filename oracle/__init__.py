@@ -180,3 +180,31 @@ def head_backward_sampled(qh, kh, vh, doh, scale, causal, rows, cols):
     dk_cols = scale * (dsc.T @ qh)
     return dq_rows, dk_cols, dv_cols
 
+
+
+def head_forward_rect(qh, kh, vh, scale, causal):
+    """Forward of one head with Nq query rows against Nk keys (decode against a
+    KV cache: explainers' glossary page, "It pairs naturally with the KV cache at
+    inference").  Causal masking is aligned to the end of the key sequence:
+    query i (0-based among the Nq) sees keys j <= Nk - Nq + i, so the Nq queries
+    are the last Nq positions of a causal sequence of length Nk.  Plain
+    definition, full rows, two-pass softmax.  Returns (O [Nq, d], LSE [Nq])."""
+    nq, nk = qh.shape[0], kh.shape[0]
+    s = scale * (qh @ kh.T)
+    if causal:
+        lim = nk - nq + np.arange(nq)[:, None]
+        s = np.where(np.arange(nk)[None, :] > lim, -np.inf, s)
+    p, m, l = _softmax_rows(s)
+    return p @ vh, m + np.log(l)
+
+
+def attention_forward_rect(q, k, v, scale, causal):
+    """O [B,H,Nq,d] and LSE [B,H,Nq] for queries q [B,H,Nq,d] against k, v [B,H,Nk,d]."""
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    B, H, Nq, d = q.shape
+    o = np.empty((B, H, Nq, v.shape[3]))
+    lse = np.empty((B, H, Nq))
+    for b in range(B):
+        for h in range(H):
+            o[b, h], lse[b, h] = head_forward_rect(q[b, h], k[b, h], v[b, h], scale, causal)
+    return o, lse
