@@ -302,7 +302,8 @@ def committed_traffic(kernel: str, workload: str):
 
 def extra_measurements(fa, torch, synth, dev, stream):
     """Single-GPU context numbers: long-sequence non-causal bf16 (fwd and bwd at
-    N=8192, d=128) and the e4m3 forward at B2 H16 N16384 d128."""
+    N=8192, d=128), the e4m3 forward at B2 H16 N16384 d128, and the split-KV
+    decode (1 and 4 queries over a 16384-key cache, 8 x 32 heads, d=128)."""
     out = {}
 
     def time_call(fn, iters=10, warm=3):
@@ -350,6 +351,23 @@ def extra_measurements(fa, torch, synth, dev, stream):
             "fp8_peak": fp8_peak, "fp8_peak_source": "2 x measured bf16 (nominal fp8:bf16 dense ratio)"}
     except Exception as e:  # noqa: BLE001
         out["fp8_fwd_b2_h16_n16384_d128"] = {"error": str(e)}
+    del q8, k8, v8, o, lse
+    # split-KV decode against a 16384-key cache: HBM-bound, K and V read once
+    # (2 GiB, well above L2, so back-to-back calls do not hit in cache)
+    B, H, Nk, d = 8, 32, 16384, 128
+    k, v = (torch.randn((B, H, Nk, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+            for _ in range(2))
+    for Nq in (1, 4):
+        q = torch.randn((B, H, Nq, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, Nq), device=dev)
+        work = torch.empty(max(16, fa.fa_fwd_decode_workspace_size(B, H, Nq, Nk, d)), dtype=torch.uint8,
+                           device=dev)
+        td = time_call(lambda: fa.fa_fwd_decode(q, k, v, o, lse, 1.0 / math.sqrt(d), True, work, stream), iters=20)
+        nbytes = 2 * B * H * Nk * d * 2 + 2 * B * H * Nq * d * 2 + B * H * Nq * 4
+        out[f"decode_b8_h32_nq{Nq}_nk16384_d128_causal"] = {
+            "us": round(td * 1e3, 2), "gbs": round(nbytes / td / 1e6, 1),
+            "frac_of_hbm": round(nbytes / td / 1e6 / peaks["hbm_gbs"], 4), "bytes": nbytes}
     return out
 
 

@@ -16,7 +16,7 @@ from ._lib import FA_OK, FAError, LIB_PATH, STATUS_CODES, STATUS_NAMES, check, l
 
 __all__ = [
     "FAError", "LIB_PATH", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size",
-    "fa_device_status",
+    "fa_device_status", "fa_fwd_decode", "fa_fwd_decode_workspace_size", "attention_decode",
     "fa_watchdog_selftest", "attention_forward", "attention_backward", "attention_forward_fp8", "lib",
     "STATUS_NAMES", "STATUS_CODES", "strerror",
 ]
@@ -96,6 +96,38 @@ def fa_bwd_deterministic(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: 
     check(lib.fa_bwd_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
                                    _ptr(dv), B, H, N, d, float(scale), int(bool(causal)), _ptr(workspace), wbytes,
                                    _stream_ptr(stream)))
+
+
+def fa_fwd_decode_workspace_size(B: int, H: int, Nq: int, Nk: int, d: int) -> int:
+    n = int(lib.fa_fwd_decode_workspace_size(B, H, Nq, Nk, d))
+    if n == ctypes.c_size_t(-1).value:
+        raise FAError(1, "invalid shape for fa_fwd_decode_workspace_size")
+    return n
+
+
+def fa_fwd_decode(q, k, v, o, lse, scale: float, causal: bool, workspace, stream=None) -> None:
+    """O, LSE <- attention of q [B,H,Nq,d] (Nq <= 16) over a KV cache k, v [B,H,Nk,d]."""
+    B, H, Nq, d = _shape(q)
+    Nk = int(k.shape[2])
+    _check_tensors((B, H, Nk, d), torch.bfloat16, k, v)
+    _check_tensors((B, H, Nq, d), torch.bfloat16, q, o)
+    _check_tensors((B, H, Nq), torch.float32, lse)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.fa_fwd_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d, float(scale),
+                            int(bool(causal)), _ptr(workspace), wbytes, _stream_ptr(stream)))
+
+
+def attention_decode(q, k, v, scale: float | None = None, causal: bool = False, workspace=None, stream=None):
+    """Allocates O, LSE (and the split workspace unless given) with torch and runs fa_fwd_decode."""
+    B, H, Nq, d = _shape(q)
+    Nk = int(k.shape[2])
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(16, fa_fwd_decode_workspace_size(B, H, Nq, Nk, d)), dtype=torch.uint8,
+                                device=q.device)
+    fa_fwd_decode(q, k, v, o, lse, _default_scale(d) if scale is None else scale, causal, workspace, stream)
+    return o, lse
 
 
 def fa_device_status(stream=None):

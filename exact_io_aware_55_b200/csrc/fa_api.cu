@@ -83,14 +83,14 @@ fa_status current_device(uint32_t** status) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // 3-D tensor map over a contiguous [BH, N, d] tensor: dims {d, N, BH},
-// box {128 bytes of d, 128 rows, 1 head}, 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap* map, const void* base, bool e4m3, int d, int N, int BH) {
+// box {128 bytes of d, box_rows rows, 1 head}, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* map, const void* base, bool e4m3, int d, int N, int BH, unsigned box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const int eb = e4m3 ? 1 : 2;
   cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
   cuuint64_t strides[2] = {cuuint64_t(d) * eb, cuuint64_t(N) * d * eb};
-  cuuint32_t box[3] = {cuuint32_t(128 / eb), 128u, 1u};
+  cuuint32_t box[3] = {cuuint32_t(128 / eb), cuuint32_t(box_rows), 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(map, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -132,6 +132,70 @@ WsLayout ws_layout(long long BH, int N, int d) {
 }
 
 fa_status launch_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH; }
+
+// Split-KV decode plan.  A head's cache is cut into items of whole 128-key
+// tiles; one persistent CTA per SM takes items round-robin, so the kernel
+// time is about (items per CTA, rounded up) x (tiles per item + a per-item
+// cost).  The per-item cost (pipeline refill, the partial result and its
+// merge, Nq d fp32 written and read back) is counted as 1/2 + Nq/64 tiles.
+// The plan takes the tiles-per-item value with the smallest such cost.  It
+// assumes 148 SMs so that the workspace size needs no device query.
+constexpr int kDecodeMaxNq = 16;
+constexpr int kDecodePlanSMs = 148;
+struct DecodePlan {
+  int n_split, tiles_per_split, tiles_per_head;
+  size_t o_off, lse_off, total;
+};
+DecodePlan decode_plan(long long BH, int Nq, int Nk, int d) {
+  DecodePlan p{};
+  const int T = (Nk + 127) / 128;
+  p.tiles_per_head = T;
+  p.tiles_per_split = T > 0 ? T : 1;
+  p.n_split = 1;
+  const double per_item = 0.5 + Nq / 64.0;
+  double best = -1.0;
+  for (int tps = 1; tps <= T; ++tps) {
+    const int ns = (T + tps - 1) / tps;
+    if ((T + ns - 1) / ns != tps) continue;          // only the balanced length for ns items
+    const long long items = BH * ns;
+    if (items > (1ll << 30)) continue;                 // item indices stay 32-bit
+    const long long rounds = (items + kDecodePlanSMs - 1) / kDecodePlanSMs;
+    const double cost = double(rounds) * (tps + per_item);
+    if (best < 0.0 || cost < best - 1e-9) {
+      best = cost;
+      p.tiles_per_split = tps;
+      p.n_split = ns;
+    }
+  }
+  const size_t parts = size_t(BH) * p.n_split * Nq;
+  p.o_off = 0;
+  p.lse_off = (parts * d * 4 + 255) / 256 * 256;
+  p.total = p.n_split > 1 ? p.lse_off + (parts * 4 + 255) / 256 * 256 : 0;
+  return p;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return kDecodePlanSMs;
+  return n > 0 ? n : kDecodePlanSMs;
+}
+
+fa_status check_decode(int B, int H, int Nq, int Nk, int d, float scale, int causal, bool* empty) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.0f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Nq > kDecodeMaxNq) return FA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > 65535) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(Nk) * d > (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  *empty = (BH == 0 || Nq == 0);
+  if (!*empty && Nk == 0) return FA_ERR_INVALID_ARG;            // queries with no keys
+  if (!*empty && causal && Nk < Nq) return FA_ERR_INVALID_ARG;  // first queries would see no key
+  return FA_OK;
+}
 
 fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                      float scale, int causal, void* stream, bool e4m3, float qd, float kd, float vd) {
@@ -253,11 +317,60 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
 
 extern "C" {
 
+size_t fa_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d) {
+  bool empty = false;
+  if (check_decode(B, H, Nq, Nk, d, 1.0f, 0, &empty) != FA_OK) return static_cast<size_t>(-1);
+  if (empty) return 0;
+  return decode_plan(static_cast<long long>(B) * H, Nq, Nk, d).total;
+}
+
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                        int Nk, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  bool empty = false;
+  fa_status st = check_decode(B, H, Nq, Nk, d, scale, causal, &empty);
+  if (st != FA_OK) return st;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  const long long BH = static_cast<long long>(B) * H;
+  const DecodePlan plan = decode_plan(BH, Nq, Nk, d);
+  if (plan.n_split > 1 && (!workspace || workspace_bytes < plan.total)) return FA_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      (workspace && !aligned(workspace, 16)))
+    return FA_ERR_ALIGNMENT;
+  uint32_t* status = nullptr;
+  if ((st = current_device(&status)) != FA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  const int bh = static_cast<int>(BH);
+  if (!make_map(&tq, q, false, d, Nq, bh, 16) || !make_map(&tk, k, false, d, Nk, bh) ||
+      !make_map(&tv, v, false, d, Nk, bh))
+    return FA_ERR_LAUNCH;
+  fa::DecodeArgs a{};
+  a.status = status;
+  a.o = o;
+  a.lse = lse;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.part_o = plan.n_split > 1 ? reinterpret_cast<float*>(ws + plan.o_off) : nullptr;
+  a.part_lse = plan.n_split > 1 ? reinterpret_cast<float*>(ws + plan.lse_off) : nullptr;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.BH = static_cast<int>(BH);
+  a.n_split = plan.n_split;
+  a.tiles_per_split = plan.tiles_per_split;
+  a.tiles_per_head = plan.tiles_per_head;
+  a.causal = causal;
+  a.c_log2 = scale * kLog2e;
+  const long long items = BH * plan.n_split;
+  const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
+  return launch_status(fa::launch_decode(tq, tk, tv, a, d, grid, static_cast<cudaStream_t>(stream)));
+}
+
 const char* fa_strerror(fa_status s) {
   switch (s) {
     case FA_OK: return "ok";
     case FA_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size, bad scale or causal flag)";
-    case FA_ERR_UNSUPPORTED: return "unsupported shape (head dimension must be 64 or 128; e4m3 needs 128)";
+    case FA_ERR_UNSUPPORTED:
+      return "unsupported shape (head dimension must be 64 or 128; e4m3 needs 128; decode takes at most 16 queries)";
     case FA_ERR_ALIGNMENT: return "misaligned pointer (tensors need 16-byte, lse 4-byte alignment)";
     case FA_ERR_ARCH: return "current CUDA device is not an sm_100 (B200-class) GPU";
     case FA_ERR_LAUNCH: return "CUDA launch or tensor-map setup failed";

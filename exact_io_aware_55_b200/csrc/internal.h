@@ -38,6 +38,18 @@ enum WaitSite : uint32_t {
   WAIT_DQ_DS = 40,
   WAIT_DQ_DSFREE = 41,
   WAIT_DQ_FINAL = 42,
+  WAIT_DEC_Q = 48,
+  WAIT_DEC_Q_EMPTY = 49,
+  WAIT_DEC_KV = 50,
+  WAIT_DEC_KV_EMPTY = 51,
+  WAIT_DEC_S = 52,
+  WAIT_DEC_S_FREE = 53,
+  WAIT_DEC_P = 54,
+  WAIT_DEC_PV = 55,
+  WAIT_DEC_RED = 56,
+  WAIT_DEC_O = 57,
+  WAIT_DEC_O_FREE = 58,
+  WAIT_DEC_STATS = 59,
   WAIT_SELFTEST = 99,
 };
 
@@ -68,6 +80,25 @@ struct BwdArgs {
   float c_log2;       // scale * log2(e)
   float scale;
 };
+
+struct DecodeArgs {
+  uint32_t* status;   // device status words (code, where)
+  void* o;            // bf16 [BH, Nq, d]
+  float* lse;         // fp32 [BH, Nq]
+  float* part_o;      // workspace: fp32 [BH, n_split, Nq, d] (normalised per split)
+  float* part_lse;    // workspace: fp32 [BH, n_split, Nq]
+  int Nq;
+  int Nk;
+  int BH;
+  int n_split;           // work items per batch-head
+  int tiles_per_split;   // 128-key tiles per item (the last item of a head may hold fewer)
+  int tiles_per_head;    // ceil(Nk / 128)
+  int causal;
+  float c_log2;          // scale * log2(e)
+};
+// q map: box {128 bytes of d, 16 rows}; k, v maps: box {128 bytes, 128 rows}.
+cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const DecodeArgs& a, int d, int grid, cudaStream_t stream);
 
 // Tensor maps: 3-D views {d, N, BH} of a [BH, N, d] tensor, box {128 bytes, 128 rows, 1},
 // 128-byte swizzle, zero fill out of bounds.

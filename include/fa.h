@@ -165,6 +165,32 @@ FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, con
 /* Size in bytes of fa_bwd_noalloc's fixed scratch array. */
 FA_API size_t fa_bwd_noalloc_max_bytes(void);
 
+/*
+ * Decode against a KV cache: Nq (1..16) new queries per (batch, head) attend
+ * over Nk cached keys ("It pairs naturally with the KV cache at inference",
+ * chipfoundryservices glossary "flash attention").  The key range is split
+ * across CTAs; each split keeps its own running max and sum, and the splits
+ * are combined by their log-sum-exp (O = sum_s exp(LSE_s - LSE) O_s).  HBM-
+ * bound: K and V are read once.
+ *   q      : in,  bf16 [B,H,Nq,d]
+ *   k, v   : in,  bf16 [B,H,Nk,d]
+ *   o      : out, bf16 [B,H,Nq,d]
+ *   lse    : out, fp32 [B,H,Nq]
+ *   causal : query i of the Nq sees keys j <= Nk - Nq + i (the queries are the
+ *            last Nq positions of the sequence); needs Nk >= Nq.
+ *   workspace : >= fa_fwd_decode_workspace_size(B,H,Nq,Nk,d) bytes of device
+ *            scratch for the per-split partial results (may be NULL when that
+ *            size is 0 or the plan uses a single split).
+ * Errors: FA_ERR_UNSUPPORTED for Nq > 16 or d not in {64,128};
+ * FA_ERR_INVALID_ARG for Nk == 0 (with queries) or causal with Nk < Nq.
+ */
+FA_API fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                               int Nq, int Nk, int d, float scale, int causal, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace fa_fwd_decode needs ((size_t)-1 for invalid arguments). */
+FA_API size_t fa_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 FA_API const char* fa_strerror(fa_status status);
 

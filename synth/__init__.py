@@ -105,6 +105,23 @@ def attention_inputs(B: int, H: int, N: int, d: int, seed: int, q_mult: float = 
     return out
 
 
+def decode_inputs(B: int, H: int, Nq: int, Nk: int, d: int, seed: int, q_mult: float = 1.0,
+                  want_f64: bool = True):
+    """Seeded bf16 inputs for decode against a KV cache: Q [B,H,Nq,d] (the
+    newest Nq positions) and K, V [B,H,Nk,d] (the cache), N(0,1) like the
+    square workloads.  Same dict layout as ``attention_inputs``."""
+    out = {"shape": (B, H, Nq, Nk, d), "seed": seed, "q_mult": q_mult, "storage": "bf16"}
+    for name, n in (("q", Nq), ("k", Nk), ("v", Nk)):
+        x = normal_f32(seed, TENSOR_IDS[name], (B, H, n, d))
+        if name == "q" and q_mult != 1.0:
+            x = x * np.float32(q_mult)
+        bits = to_bf16_bits(x)
+        out[name + "_bits"] = bits
+        if want_f64:
+            out[name] = bf16_bits_to_f64(bits)
+    return out
+
+
 def head_f64(inp, name: str, b: int, h: int) -> np.ndarray:
     """Exact float64 values of one head of tensor ``name``."""
     bits = inp[name + "_bits"][b, h]

@@ -89,3 +89,58 @@ def test_noalloc_limit_is_checked_first():
     st = fa.lib.fa_bwd_noalloc(*([4096] * 9), 1, 32, 4096, 128, F(0.1), 0, None)
     assert st == C["FA_ERR_SCRATCH_LIMIT"]
     assert fa.lib.fa_bwd_noalloc(*([4096] * 9), 1, 1, 16, 96, F(0.1), 0, None) == C["FA_ERR_UNSUPPORTED"]
+
+
+def decode_plan(B, H, Nq, Nk, d):
+    """Items per head and workspace bytes of the decode path: a head's cache is
+    cut into items of whole 128-key tiles; with one persistent CTA per SM (148
+    SMs) the time is about ceil(items / 148) x (tiles per item + 1/2 + Nq/64),
+    and the balanced tiles-per-item value with the smallest such cost wins."""
+    BH, T = B * H, -(-Nk // 128)
+    best, plan = None, (1, max(T, 1))
+    for tps in range(1, T + 1):
+        ns = -(-T // tps)
+        if -(-T // ns) != tps or BH * ns > 1 << 30:
+            continue
+        cost = -(-(BH * ns) // 148) * (tps + 0.5 + Nq / 64)
+        if best is None or cost < best - 1e-9:
+            best, plan = cost, (ns, tps)
+    ns = plan[0]
+    parts = BH * ns * Nq
+    total = (parts * d * 4 + 255) // 256 * 256 + (parts * 4 + 255) // 256 * 256 if ns > 1 else 0
+    return ns, total
+
+
+def test_decode_workspace_size_formula():
+    for shape in [(1, 1, 1, 64, 64), (1, 1, 1, 4096, 128), (8, 32, 1, 16384, 128), (2, 3, 16, 1000, 64),
+                  (1, 1, 5, 70000, 128), (64, 32, 1, 4096, 128)]:
+        assert fa.fa_fwd_decode_workspace_size(*shape) == decode_plan(*shape)[1]
+    assert decode_plan(1, 1, 1, 64, 64) == (1, 0)                # one tile: one item, no workspace
+    assert decode_plan(1, 1, 1, 4096 * 37, 128)[0] == 148        # one head: an item per SM
+    assert decode_plan(8, 32, 1, 16384, 128)[0] == 4             # 1024 items of 32 tiles
+    assert decode_plan(64, 32, 1, 4096, 128)[0] == 1             # enough heads: no split
+    assert fa.fa_fwd_decode_workspace_size(1, 1, 0, 64, 64) == 0
+    with pytest.raises(fa.FAError):
+        fa.fa_fwd_decode_workspace_size(1, 1, 17, 64, 64)
+    with pytest.raises(fa.FAError):
+        fa.fa_fwd_decode_workspace_size(1, 1, 1, 64, 96)
+
+
+def test_decode_argument_errors_launch_nothing():
+    p = 4096
+
+    def dec(Nq=1, Nk=64, d=64, causal=0, ws=None, wbytes=0, q=p, o=p, lse=p, scale=0.125):
+        return fa.lib.fa_fwd_decode(q, p, p, o, lse, 1, 1, Nq, Nk, d, F(scale), causal, ws, wbytes, None)
+
+    assert dec(Nq=17) == C["FA_ERR_UNSUPPORTED"]
+    assert dec(d=96) == C["FA_ERR_UNSUPPORTED"]
+    assert dec(Nk=0) == C["FA_ERR_INVALID_ARG"]                     # queries with nothing to attend to
+    assert dec(Nq=8, Nk=4, causal=1) == C["FA_ERR_INVALID_ARG"]     # causal needs Nk >= Nq
+    assert dec(scale=-1.0) == C["FA_ERR_INVALID_ARG"]
+    assert dec(q=None) == C["FA_ERR_INVALID_ARG"]
+    assert dec(q=p + 8) == C["FA_ERR_ALIGNMENT"]
+    assert dec(Nk=4096) == C["FA_ERR_WORKSPACE"]                    # 16 splits need a workspace
+    need = fa.fa_fwd_decode_workspace_size(1, 1, 1, 4096, 64)
+    assert dec(Nk=4096, ws=p, wbytes=need - 1) == C["FA_ERR_WORKSPACE"]
+    assert dec(Nk=4096, ws=p + 4, wbytes=need) == C["FA_ERR_ALIGNMENT"]
+    assert dec(Nq=0, q=None, o=None, lse=None) == C["FA_OK"]        # empty: nothing to do
