@@ -133,8 +133,9 @@ WsLayout ws_layout(long long BH, int N, int d) {
 
 fa_status launch_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH; }
 
-// Split-KV decode plan.  A head's cache is cut into items of whole 128-key
-// tiles; one persistent CTA per SM takes items round-robin, so the kernel
+// Split-KV decode plan.  A head's cache is cut into items of whole key tiles
+// (128 keys at d = 128, 256 at d = 64: 64 KB of K and V per tile either way);
+// one persistent CTA per SM takes items round-robin, so the kernel
 // time is about (items per CTA, rounded up) x (tiles per item + a per-item
 // cost).  The per-item cost (pipeline refill, the partial result and its
 // merge, Nq d fp32 written and read back) is counted as 1/2 + Nq/64 tiles.
@@ -148,7 +149,8 @@ struct DecodePlan {
 };
 DecodePlan decode_plan(long long BH, int Nq, int Nk, int d) {
   DecodePlan p{};
-  const int T = (Nk + 127) / 128;
+  const int tile_keys = d == 64 ? 256 : 128;
+  const int T = (Nk + tile_keys - 1) / tile_keys;
   p.tiles_per_head = T;
   p.tiles_per_split = T > 0 ? T : 1;
   p.n_split = 1;

@@ -2,12 +2,13 @@
 //
 // The glossary page (chipfoundryservices "flash attention", last section)
 // pairs the method with the KV cache at inference.  Each (batch-head) cache is
-// cut into splits of whole 128-key tiles; a split is one work item, and the
+// cut into splits of whole key tiles (128 keys at d = 128, 256 at d = 64, so
+// that a tile of K and V is 64 KB either way); a split is one work item, and the
 // persistent CTAs (one per SM) take items round-robin.  Per item the online
 // softmax runs over the split's tiles exactly as in the square forward, but
-// with the product transposed so that the 128 keys of a tile fill the MMA's
-// M dimension and the (padded) 16 queries its N dimension:
-//   S^T = K_j Q^T        128 x 16 fp32 in TMEM       (tcgen05, both K-major)
+// with the product transposed so that the keys of a tile fill the MMA's M
+// dimension (one 128-key MMA per sub-tile) and the (padded) 16 queries its N:
+//   S^T = K_j Q^T        keys x 16 fp32 in TMEM      (tcgen05, both K-major)
 //   P^T = exp2(S^T * scale * log2 e - m)   thread = key; the max over the
 //                        tile's keys is a warp redux and a four-warp exchange
 //   O^T += V_j^T P^T     d x 16 fp32 in TMEM          (A = V tile MN-major,
@@ -32,7 +33,6 @@ namespace fa {
 
 namespace {
 
-constexpr int kDecTile = 128;      // keys per tile = MMA M of S^T
 constexpr int kDecNq = 16;         // query columns = MMA N (Nq <= 16, rest zero)
 constexpr int kDecThreads = 384;
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -40,17 +40,21 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 template <int D>
 struct DecShape {
-  static constexpr int kTileBytes = kDecTile * D * 2;     // one K (or V) tile
+  static constexpr int kSub = (D == 64) ? 2 : 1;          // 128-key sub-tiles per tile
+  static constexpr int kTileKeys = 128 * kSub;
+  static constexpr int kTileBytes = kTileKeys * D * 2;    // K (or V) of one tile: 32 KB
   static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
-  static constexpr int kNS = (D == 128) ? 3 : 6;          // ring depth: 192 KB either way
+  static constexpr int kNS = 3;                           // ring depth: 192 KB
   static constexpr int kQBytes = kDecNq * D * 2;          // 16 query rows
-  static constexpr int kPBytes = kDecNq * kDecTile * 2;   // P^T of one tile
-  static constexpr int kChunks = D / 64;                  // 128-byte column chunks
-  static constexpr int kKSteps = D / 16;
+  static constexpr int kPBytes = kDecNq * kTileKeys * 2;  // P^T of one tile
+  static constexpr int kChunks = D / 64;                  // 128-byte column chunks (16 KB per sub-tile)
+  static constexpr int kKSteps = D / 16;                  // S^T k-steps per sub-tile
+  static constexpr int kPvSteps = kTileKeys / 16;         // O^T k-steps per tile
   static constexpr uint32_t kIdS = idesc_bf16(128, kDecNq, false, false);   // S^T = K Q^T
   static constexpr uint32_t kIdO = idesc_bf16(D, kDecNq, true, false);      // O^T = V^T P^T
-  static constexpr uint32_t kColS = 0;    // S^T buffers at columns 0, 16
-  static constexpr uint32_t kColO = 32;   // O^T buffers at columns 32, 48
+  static constexpr uint32_t kColS = 0;                    // two S^T buffers of 16 * kSub columns
+  static constexpr uint32_t kColO = 32 * kSub;            // two O^T buffers of 16 columns
+  static constexpr uint32_t kTmemCols = (kColO + 32 <= 64) ? 64 : 128;
 };
 
 template <int NS>
@@ -139,7 +143,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&b->tmem_base, 64);
+    tmem_alloc(&b->tmem_base, S::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -169,14 +173,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           ok = false;
           break;
         }
-        const int key0 = (w.t0 + j) * kDecTile;
+        const int key0 = (w.t0 + j) * S::kTileKeys;
         uint8_t* st = sKV + s * S::kStageBytes;
         mbar_arrive_expect_tx_e(&b->kv_full[s], S::kStageBytes);
 #pragma unroll
-        for (int c = 0; c < S::kChunks; ++c) {
-          tma_load_3d_hint_e(st + c * 16384, &tmK, &b->kv_full[s], c * 64, key0, w.bh, pol);
-          tma_load_3d_hint_e(st + S::kTileBytes + c * 16384, &tmV, &b->kv_full[s], c * 64, key0, w.bh, pol);
-        }
+        for (int u = 0; u < S::kSub; ++u)
+#pragma unroll
+          for (int c = 0; c < S::kChunks; ++c) {
+            const int off = (u * S::kChunks + c) * 16384;
+            tma_load_3d_hint_e(st + off, &tmK, &b->kv_full[s], c * 64, key0 + 128 * u, w.bh, pol);
+            tma_load_3d_hint_e(st + S::kTileBytes + off, &tmV, &b->kv_full[s], c * 64, key0 + 128 * u, w.bh, pol);
+          }
       }
     }
   } else if (warp == 1) {
@@ -195,8 +202,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       tc_fence_after();
       const int s = gg % NS;
 #pragma unroll
-      for (int kt = 0; kt < 8; ++kt) {
-        const uint64_t va = uint64_t((s * S::kStageBytes + kt * 2048) >> 4);
+      for (int kt = 0; kt < S::kPvSteps; ++kt) {
+        const uint64_t va = uint64_t((s * S::kStageBytes + (kt >> 3) * S::kChunks * 16384 + (kt & 7) * 2048) >> 4);
         const uint64_t pb_off = uint64_t((pb * S::kPBytes + (kt >> 2) * 2048 + (kt & 3) * 32) >> 4);
         mma_f16_ss_e(tmem + S::kColO + 16 * ob, dV + va, dP + pb_off, S::kIdO, (!first || kt > 0) ? 1u : 0u);
       }
@@ -217,11 +224,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < S::kKSteps; ++ks) {
-          const uint64_t ka = uint64_t((s * S::kStageBytes + (ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
-          const uint64_t qo = uint64_t((qb * S::kQBytes + (ks >> 2) * 2048 + (ks & 3) * 32) >> 4);
-          mma_f16_ss_e(tmem + S::kColS + 16 * sb, dK + ka, dQ + qo, S::kIdS, ks > 0 ? 1u : 0u);
-        }
+        for (int u = 0; u < S::kSub; ++u)
+#pragma unroll
+          for (int ks = 0; ks < S::kKSteps; ++ks) {
+            const uint64_t ka = uint64_t((s * S::kStageBytes + (u * S::kChunks + (ks >> 2)) * 16384 + (ks & 3) * 32) >> 4);
+            const uint64_t qo = uint64_t((qb * S::kQBytes + (ks >> 2) * 2048 + (ks & 3) * 32) >> 4);
+            mma_f16_ss_e(tmem + S::kColS + 16 * (sb * S::kSub + u), dK + ka, dQ + qo, S::kIdS, ks > 0 ? 1u : 0u);
+          }
         tc_commit_e(&b->s_full[sb]);
         if (j == w.nt - 1) tc_commit_e(&b->q_empty[qb]);
         if (j > 0 && !issue_pv(g - 1, ob, j == 1)) {
@@ -256,29 +265,39 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           break;
         }
         tc_fence_after();
-        float s[kDecNq];
-        {
+        constexpr int U = S::kSub;
+        float s[U][kDecNq];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
           uint32_t r[16];
-          tmem_ld_x16(lane_base + S::kColS + 16 * sb, r);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&b->s_free[sb]);
+          tmem_ld_x16(lane_base + S::kColS + 16 * (sb * U + u), r);
 #pragma unroll
-          for (int q = 0; q < kDecNq; ++q) s[q] = __uint_as_float(r[q]) * cl;
+          for (int q = 0; q < kDecNq; ++q) s[u][q] = __uint_as_float(r[q]) * cl;
         }
-        const int tile0 = (w.t0 + j) * kDecTile;
-        const int key = tile0 + wq * 32 + lane;
-        if (tile0 + kDecTile > Nk || (a.causal && tile0 + kDecTile - 1 > Nk - Nq)) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b->s_free[sb]);
+        const int tile0 = (w.t0 + j) * S::kTileKeys;
+        if (tile0 + S::kTileKeys > Nk || (a.causal && tile0 + S::kTileKeys - 1 > Nk - Nq)) {
 #pragma unroll
-          for (int q = 0; q < kDecNq; ++q)
-            if (key >= Nk || (a.causal && key > Nk - Nq + q)) s[q] = -INFINITY;
+          for (int u = 0; u < U; ++u) {
+            const int key = tile0 + 128 * u + wq * 32 + lane;
+#pragma unroll
+            for (int q = 0; q < kDecNq; ++q)
+              if (key >= Nk || (a.causal && key > Nk - Nq + q)) s[u][q] = -INFINITY;
+          }
         }
         // tile maximum per query: warp redux, then the four softmax warps
         float* rm = &b->red_max[g & 1][wq][0];
         {
           float wm[kDecNq];
 #pragma unroll
-          for (int q = 0; q < kDecNq; ++q) wm[q] = redux_max(s[q]);
+          for (int q = 0; q < kDecNq; ++q) {
+            float x = s[0][q];
+#pragma unroll
+            for (int u = 1; u < U; ++u) x = fmaxf(x, s[u][q]);
+            wm[q] = redux_max(x);
+          }
           if (lane == 0) {
 #pragma unroll
             for (int q = 0; q < kDecNq; q += 4)
@@ -332,20 +351,21 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             tmem_wait_st();
           }
         }
-        // P^T into shared memory: B operand, K-major, rows = queries, 128 keys
-        // in two 64-key chunks of 128-byte swizzled rows.
+        // P^T into shared memory: B operand, K-major, rows = queries, the
+        // tile's keys in 64-key chunks of 128-byte swizzled rows.
         const int pb = g & 1;
         if (g >= 2 && !mbar_wait_warp(&b->pv_done[pb], ((g - 2) >> 1) & 1, wc, WAIT_DEC_PV)) {
           ok = false;
           break;
         }
-        {
-          const int kk = wq * 32 + lane;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int kk = 128 * u + wq * 32 + lane;
           uint8_t* pbase = sP + pb * S::kPBytes + (kk >> 6) * 2048 + (kk & 7) * 2;
           const int unit = (kk & 63) >> 3;
 #pragma unroll
           for (int q = 0; q < kDecNq; ++q) {
-            const float p = (s[q] == -INFINITY) ? 0.0f : ex2_approx(s[q] - m_used[q]);
+            const float p = (s[u][q] == -INFINITY) ? 0.0f : ex2_approx(s[u][q] - m_used[q]);
             l_t[q] += p;
             *reinterpret_cast<__nv_bfloat16*>(pbase + (q >> 3) * 1024 + (q & 7) * 128 + ((unit ^ (q & 7)) << 4)) =
                 __float2bfloat16_rn(p);
@@ -428,32 +448,54 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, S::kTmemCols);
   }
 }
 
-// O = sum_s exp(LSE_s - LSE) O_s with LSE = log sum_s exp(LSE_s), per
-// (batch-head, query, column); one block per batch-head.
+// O = sum_s exp(LSE_s - LSE) O_s with LSE = log sum_s exp(LSE_s).  One block
+// per (query, batch-head); thread = (output column, one of kParts interleaved
+// subsets of the splits), the subsets summed through shared memory.
+constexpr int kMergeThreads = 256;
+
 template <int D>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
-  const int bh = blockIdx.x;
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const DecodeArgs a) {
+  constexpr int kParts = kMergeThreads / D;
+  __shared__ float red[kMergeThreads / 32];
+  __shared__ float acc_s[kParts][D];
+  __shared__ float l_s[kParts];
+  const int q = blockIdx.x, bh = blockIdx.y;
   const int Nq = a.Nq, ns = a.n_split;
-  for (int idx = threadIdx.x; idx < Nq * D; idx += blockDim.x) {
-    const int qi = idx / D, c = idx - qi * D;
-    const float* pl = a.part_lse + size_t(bh) * ns * Nq + qi;
-    float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, pl[size_t(s) * Nq]);
-    float L = 0.0f, acc = 0.0f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < ns; ++s) {
-        const float w = __expf(pl[size_t(s) * Nq] - M);
-        L += w;
-        acc = fmaf(w, a.part_o[((size_t(bh) * ns + s) * Nq + qi) * D + c], acc);
-      }
+  const int c = threadIdx.x % D, part = threadIdx.x / D;
+  const float* pl = a.part_lse + size_t(bh) * ns * Nq + q;            // split stride Nq
+  const float* po = a.part_o + (size_t(bh) * ns * Nq + q) * D + c;    // split stride Nq * D
+  float m = -INFINITY;
+  for (int s = threadIdx.x; s < ns; s += kMergeThreads) m = fmaxf(m, pl[size_t(s) * Nq]);
+  m = redux_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kMergeThreads / 32; ++w) m = fmaxf(m, red[w]);
+  float L = 0.0f, acc = 0.0f;
+  if (m != -INFINITY) {
+#pragma unroll 4
+    for (int s = part; s < ns; s += kParts) {
+      const float wgt = __expf(pl[size_t(s) * Nq] - m);
+      L += wgt;
+      acc = fmaf(wgt, po[size_t(s) * Nq * D], acc);
     }
-    reinterpret_cast<__nv_bfloat16*>(a.o)[(size_t(bh) * Nq + qi) * D + c] =
-        __float2bfloat16_rn(L > 0.0f ? acc / L : 0.0f);
-    if (c == 0) a.lse[size_t(bh) * Nq + qi] = (L > 0.0f) ? M + __logf(L) : -INFINITY;
+  }
+  acc_s[part][c] = acc;
+  if (c == 0) l_s[part] = L;
+  __syncthreads();
+  if (part == 0) {
+    float at = 0.0f, lt = 0.0f;
+#pragma unroll
+    for (int p = 0; p < kParts; ++p) {
+      at += acc_s[p][c];
+      lt += l_s[p];
+    }
+    reinterpret_cast<__nv_bfloat16*>(a.o)[(size_t(bh) * Nq + q) * D + c] = __float2bfloat16_rn(lt > 0.0f ? at / lt : 0.0f);
+    if (c == 0) a.lse[size_t(bh) * Nq + q] = (lt > 0.0f) ? m + __logf(lt) : -INFINITY;
   }
 }
 
@@ -468,7 +510,7 @@ cudaError_t launch_decode_t(const CUtensorMap& tq, const CUtensorMap& tk, const 
   kern<<<grid, kDecThreads, smem, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.n_split == 1) return e;
-  decode_merge_kernel<D><<<a.BH, 128, 0, stream>>>(a);
+  decode_merge_kernel<D><<<dim3(a.Nq, a.BH), kMergeThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -93,10 +93,11 @@ def test_noalloc_limit_is_checked_first():
 
 def decode_plan(B, H, Nq, Nk, d):
     """Items per head and workspace bytes of the decode path: a head's cache is
-    cut into items of whole 128-key tiles; with one persistent CTA per SM (148
-    SMs) the time is about ceil(items / 148) x (tiles per item + 1/2 + Nq/64),
-    and the balanced tiles-per-item value with the smallest such cost wins."""
-    BH, T = B * H, -(-Nk // 128)
+    cut into items of whole key tiles (128 keys at d=128, 256 at d=64); with
+    one persistent CTA per SM (148 SMs) the time is about ceil(items / 148) x
+    (tiles per item + 1/2 + Nq/64), and the balanced tiles-per-item value with
+    the smallest such cost wins."""
+    BH, T = B * H, -(-Nk // (256 if d == 64 else 128))
     best, plan = None, (1, max(T, 1))
     for tps in range(1, T + 1):
         ns = -(-T // tps)
