@@ -282,6 +282,64 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_case(args):
+    """One named path on --shape, for profiling (a short JSON line, not the
+    bench line): 'decode' (B,H,Nk,d with --nq queries, causal) or 'standard'
+    (B,H,N,d: the materialising baseline, then the fused forward, per step)."""
+    import torch
+
+    import exact_io_aware_55_b200 as fa
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    B, H, N, d = (int(x) for x in args.shape.split(","))
+
+    def rnd(*shape):
+        return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    if args.case == "decode":
+        q, k, v = rnd(B, H, args.nq, d), rnd(B, H, N, d), rnd(B, H, N, d)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, args.nq), device=dev)
+        work = torch.empty(max(16, fa.fa_fwd_decode_workspace_size(B, H, args.nq, N, d)), dtype=torch.uint8,
+                           device=dev)
+
+        def step():
+            fa.fa_fwd_decode(q, k, v, o, lse, d ** -0.5, True, work, stream)
+        nbytes = 4 * B * H * N * d
+    else:
+        q, k, v = rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), device=dev)
+        work = torch.empty(fa.fa_fwd_standard_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+
+        def step():
+            fa.fa_fwd_standard(q, k, v, o, lse, d ** -0.5, args.causal, work, stream)
+            fa.fa_fwd(q, k, v, o, lse, d ** -0.5, args.causal, stream)
+        nbytes = None
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st, where = fa.fa_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} (wait site {where})")
+    ms = e0.elapsed_time(e1) / args.steps
+    line = {"case": args.case, "shape": args.shape, "ms_per_step": round(ms, 5)}
+    if nbytes:
+        line["nq"] = args.nq
+        line["gbs"] = round(nbytes / ms / 1e6, 1)
+    print(json.dumps(line), flush=True)
+
+
 def committed_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the library build that is loaded now (same source digest); else None."""
@@ -302,7 +360,8 @@ def committed_traffic(kernel: str, workload: str):
 
 def extra_measurements(fa, torch, synth, dev, stream):
     """Single-GPU context numbers: long-sequence non-causal bf16 (fwd and bwd at
-    N=8192, d=128), the e4m3 forward at B2 H16 N16384 d128, and the split-KV
+    N=8192, d=128), the e4m3 forward at B2 H16 N16384 d128, standard
+    (materialising) attention against the fused forward, and the split-KV
     decode (1 and 4 queries over a 16384-key cache, 8 x 32 heads, d=128)."""
     out = {}
 
@@ -352,6 +411,25 @@ def extra_measurements(fa, torch, synth, dev, stream):
     except Exception as e:  # noqa: BLE001
         out["fp8_fwd_b2_h16_n16384_d128"] = {"error": str(e)}
     del q8, k8, v8, o, lse
+    # standard (materialising) attention against the fused forward on the same
+    # inputs: the IO claim of the method, measured
+    for (B, H, N, d) in ((4, 16, 2048, 64), (1, 32, 8192, 128)):
+        q, k, v = (torch.randn((B, H, N, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+                   for _ in range(3))
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), device=dev)
+        work = torch.empty(fa.fa_fwd_standard_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+        sc = 1.0 / math.sqrt(d)
+        ts = time_call(lambda: fa.fa_fwd_standard(q, k, v, o, lse, sc, False, work, stream))
+        tf = time_call(lambda: fa.fa_fwd(q, k, v, o, lse, sc, False, stream))
+        Np = -(-N // 128) * 128
+        F = fwd_flops(B, H, N, d, False)
+        out[f"standard_vs_fused_b{B}_h{H}_n{N}_d{d}"] = {
+            "standard_ms": round(ts, 4), "fused_ms": round(tf, 4), "speedup": round(ts / tf, 2),
+            "standard_tflops": round(F / ts / 1e9, 1), "fused_tflops": round(F / tf / 1e9, 1),
+            "standard_hbm_bytes": B * H * (12 * N * Np + 8 * N * d),
+            "fused_hbm_bytes": B * H * (8 * N * d + 4 * N)}
+        del q, k, v, o, lse, work
     # split-KV decode against a 16384-key cache: HBM-bound, K and V read once
     # (2 GiB, well above L2, so back-to-back calls do not hit in cache)
     B, H, Nk, d = 8, 32, 16384, 128
@@ -450,9 +528,17 @@ def main():
     ap.add_argument("--ref-step-budget", type=float, default=1.0)
     ap.add_argument("--shape", default="", help="B,H,N,d of another workload (default: the bench workload)")
     ap.add_argument("--causal", action="store_true")
+    ap.add_argument("--case", choices=["decode", "standard"], default="",
+                    help="profile one path on --shape instead of the bench step")
+    ap.add_argument("--nq", type=int, default=1, help="queries per head for --case decode")
     ap.add_argument("--clock-window", type=float, default=1.5,
                     help="seconds of steps run under the clock sampler before the timed region")
     args = ap.parse_args()
+    if args.case:
+        if not args.shape:
+            ap.error("--case needs --shape")
+        run_case(args)
+        return
     apply_shape(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

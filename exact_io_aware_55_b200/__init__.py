@@ -17,6 +17,7 @@ from ._lib import FA_OK, FAError, LIB_PATH, STATUS_CODES, STATUS_NAMES, check, l
 __all__ = [
     "FAError", "LIB_PATH", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size",
     "fa_device_status", "fa_fwd_decode", "fa_fwd_decode_workspace_size", "attention_decode",
+    "fa_fwd_standard", "fa_fwd_standard_workspace_size", "attention_forward_standard",
     "fa_watchdog_selftest", "attention_forward", "attention_backward", "attention_forward_fp8", "lib",
     "STATUS_NAMES", "STATUS_CODES", "strerror",
 ]
@@ -127,6 +128,35 @@ def attention_decode(q, k, v, scale: float | None = None, causal: bool = False, 
         workspace = torch.empty(max(16, fa_fwd_decode_workspace_size(B, H, Nq, Nk, d)), dtype=torch.uint8,
                                 device=q.device)
     fa_fwd_decode(q, k, v, o, lse, _default_scale(d) if scale is None else scale, causal, workspace, stream)
+    return o, lse
+
+
+def fa_fwd_standard_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    n = int(lib.fa_fwd_standard_workspace_size(B, H, N, d))
+    if n == ctypes.c_size_t(-1).value:
+        raise FAError(1, "invalid shape for fa_fwd_standard_workspace_size")
+    return n
+
+
+def fa_fwd_standard(q, k, v, o, lse, scale: float, causal: bool, workspace, stream=None) -> None:
+    """Standard attention with S and P materialised in the workspace (the IO baseline)."""
+    B, H, N, d = _shape(q)
+    _check_tensors((B, H, N, d), torch.bfloat16, q, k, v, o)
+    _check_tensors((B, H, N), torch.float32, lse)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.fa_fwd_standard(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                              int(bool(causal)), _ptr(workspace), wbytes, _stream_ptr(stream)))
+
+
+def attention_forward_standard(q, k, v, scale: float | None = None, causal: bool = False, workspace=None,
+                               stream=None):
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(256, fa_fwd_standard_workspace_size(B, H, N, d)), dtype=torch.uint8,
+                                device=q.device)
+    fa_fwd_standard(q, k, v, o, lse, _default_scale(d) if scale is None else scale, causal, workspace, stream)
     return o, lse
 
 

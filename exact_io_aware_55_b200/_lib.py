@@ -54,6 +54,10 @@ def _load() -> ctypes.CDLL:
     lib.fa_fwd_decode.restype = i
     lib.fa_fwd_decode_workspace_size.argtypes = [i, i, i, i, i]
     lib.fa_fwd_decode_workspace_size.restype = sz
+    lib.fa_fwd_standard.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_fwd_standard.restype = i
+    lib.fa_fwd_standard_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_fwd_standard_workspace_size.restype = sz
     lib.fa_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_bwd_deterministic.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]

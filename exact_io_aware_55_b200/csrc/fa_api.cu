@@ -99,6 +99,21 @@ bool make_map(CUtensorMap* map, const void* base, bool e4m3, int d, int N, int B
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over the standard path's probabilities P [BH, N, Np] bf16:
+// dims {Np, N, BH}, box {64 columns, 128 rows, 1 head}, 128-byte swizzle.
+bool make_map_p(CUtensorMap* map, const void* base, int Np, int N, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(Np), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(Np) * 2, cuuint64_t(N) * Np * 2};
+  cuuint32_t box[3] = {64u, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Shape checks shared by every entry point.  Sets *empty when there is
 // nothing to compute.
 fa_status check_shape(int B, int H, int N, int d, float scale, int causal, bool* empty) {
@@ -365,6 +380,61 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
   const long long items = BH * plan.n_split;
   const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
   return launch_status(fa::launch_decode(tq, tk, tv, a, d, grid, static_cast<cudaStream_t>(stream)));
+}
+
+// Standard attention workspace: S fp32 [BH, N, Np] then P bf16 [BH, N, Np].
+struct StdLayout {
+  size_t p_off, total;
+};
+StdLayout std_layout(long long BH, int N) {
+  const size_t cells = size_t(BH) * N * padded_rows(N);
+  StdLayout w{};
+  w.p_off = (cells * 4 + 255) / 256 * 256;
+  w.total = w.p_off + cells * 2;
+  return w;
+}
+
+size_t fa_fwd_standard_workspace_size(int B, int H, int N, int d) {
+  bool empty = false;
+  if (check_shape(B, H, N, d, 1.0f, 0, &empty) != FA_OK) return static_cast<size_t>(-1);
+  if (empty) return 0;
+  return std_layout(static_cast<long long>(B) * H, N).total;
+}
+
+fa_status fa_fwd_standard(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                          int d, float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  bool empty = false;
+  fa_status st = check_shape(B, H, N, d, scale, causal, &empty);
+  if (st != FA_OK) return st;
+  if (empty) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  const long long BH = static_cast<long long>(B) * H;
+  const StdLayout w = std_layout(BH, N);
+  if (!workspace || workspace_bytes < w.total) return FA_ERR_WORKSPACE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(workspace, 256))
+    return FA_ERR_ALIGNMENT;
+  uint32_t* status = nullptr;
+  if ((st = current_device(&status)) != FA_OK) return st;
+  const int bh = static_cast<int>(BH);
+  const int Np = static_cast<int>(padded_rows(N));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  CUtensorMap tq, tk, tv, tp;
+  if (!make_map(&tq, q, false, d, N, bh) || !make_map(&tk, k, false, d, N, bh) || !make_map(&tv, v, false, d, N, bh) ||
+      !make_map_p(&tp, ws + w.p_off, Np, N, bh))
+    return FA_ERR_LAUNCH;
+  fa::StdArgs a{};
+  a.status = status;
+  a.s = reinterpret_cast<float*>(ws);
+  a.p = reinterpret_cast<__nv_bfloat16*>(ws + w.p_off);
+  a.o = o;
+  a.lse = lse;
+  a.N = N;
+  a.Np = Np;
+  a.BH = bh;
+  a.causal = causal;
+  a.scale = scale;
+  return launch_status(fa::launch_standard(tq, tk, tv, tp, a, d, static_cast<cudaStream_t>(stream)));
 }
 
 const char* fa_strerror(fa_status s) {

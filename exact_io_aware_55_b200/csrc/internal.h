@@ -1,6 +1,7 @@
 // Internal launch interface between the C ABI (fa_api.cu) and the kernels.
 #pragma once
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -50,6 +51,11 @@ enum WaitSite : uint32_t {
   WAIT_DEC_O = 57,
   WAIT_DEC_O_FREE = 58,
   WAIT_DEC_STATS = 59,
+  WAIT_STD_LOAD = 64,
+  WAIT_STD_MMA = 65,
+  WAIT_STD_PV_EMPTY = 66,
+  WAIT_STD_PV_FULL = 67,
+  WAIT_STD_PV_DONE = 68,
   WAIT_SELFTEST = 99,
 };
 
@@ -96,6 +102,22 @@ struct DecodeArgs {
   int causal;
   float c_log2;          // scale * log2(e)
 };
+struct StdArgs {
+  uint32_t* status;   // device status words (code, where)
+  float* s;           // workspace: fp32 [BH, N, Np] scores (already scaled)
+  __nv_bfloat16* p;   // workspace: bf16 [BH, N, Np] probabilities
+  void* o;            // bf16 [BH, N, d]
+  float* lse;         // fp32 [BH, N]
+  int N;
+  int Np;             // N rounded up to 128
+  int BH;
+  int causal;
+  float scale;
+};
+// p map: dims {Np, N, BH}, box {64 columns, 128 rows}.
+cudaError_t launch_standard(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tp, const StdArgs& a, int d, cudaStream_t stream);
+
 // q map: box {128 bytes of d, 16 rows}; k, v maps: box {128 bytes, 128 rows}.
 cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const DecodeArgs& a, int d, int grid, cudaStream_t stream);

@@ -191,6 +191,26 @@ FA_API fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void
 /* Bytes of workspace fa_fwd_decode needs ((size_t)-1 for invalid arguments). */
 FA_API size_t fa_fwd_decode_workspace_size(int B, int H, int Nq, int Nk, int d);
 
+/*
+ * Standard (materialising) attention, the baseline the method is measured
+ * against (explainers.rudrite.com "flash-attention-anatomy", Q&A "Why is
+ * attention memory-bound, and how does FlashAttention fix it?": S is written
+ * to HBM, read back for the softmax, P written, and read again for P V).
+ * Same arguments and results as fa_fwd (O bf16, LSE fp32 natural log, causal
+ * top-left aligned), computed in three passes through the workspace:
+ *   S = scale Q K^T   fp32 [B,H,N,Np]   (Np = N rounded up to 128)
+ *   P = softmax(S)    bf16 [B,H,N,Np]   (normalised; causal mask applied here)
+ *   O = P V
+ * workspace: >= fa_fwd_standard_workspace_size(B,H,N,d) bytes of device
+ * memory, 256-byte aligned; about 6 N^2 bytes per head.
+ */
+FA_API fa_status fa_fwd_standard(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                 int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/* Bytes of workspace fa_fwd_standard needs ((size_t)-1 for invalid arguments). */
+FA_API size_t fa_fwd_standard_workspace_size(int B, int H, int N, int d);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 FA_API const char* fa_strerror(fa_status status);
 

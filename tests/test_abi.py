@@ -145,3 +145,25 @@ def test_decode_argument_errors_launch_nothing():
     assert dec(Nk=4096, ws=p, wbytes=need - 1) == C["FA_ERR_WORKSPACE"]
     assert dec(Nk=4096, ws=p + 4, wbytes=need) == C["FA_ERR_ALIGNMENT"]
     assert dec(Nq=0, q=None, o=None, lse=None) == C["FA_OK"]        # empty: nothing to do
+
+
+def test_standard_workspace_and_errors():
+    # S fp32 then P bf16, both [B,H,N,Np] with Np = N rounded up to 128; S rounded up to 256 bytes
+    def expect(B, H, N, d):
+        cells = B * H * N * (-(-N // 128) * 128)
+        return (cells * 4 + 255) // 256 * 256 + cells * 2
+    for shape in [(1, 1, 1, 64), (2, 3, 300, 128), (4, 16, 2048, 64)]:
+        assert fa.fa_fwd_standard_workspace_size(*shape) == expect(*shape)
+    assert fa.fa_fwd_standard_workspace_size(1, 1, 0, 64) == 0
+    p = 4096
+    need = fa.fa_fwd_standard_workspace_size(1, 1, 64, 64)
+
+    def std(ws=p, wbytes=need, d=64, q=p):
+        return fa.lib.fa_fwd_standard(q, p, p, p, p, 1, 1, 64, d, F(0.125), 0, ws, wbytes, None)
+
+    assert std(ws=None, wbytes=0) == C["FA_ERR_WORKSPACE"]
+    assert std(wbytes=need - 1) == C["FA_ERR_WORKSPACE"]
+    assert std(ws=p + 16) == C["FA_ERR_ALIGNMENT"]            # workspace must be 256-byte aligned
+    assert std(q=p + 8) == C["FA_ERR_ALIGNMENT"]
+    assert std(d=96) == C["FA_ERR_UNSUPPORTED"]
+    assert std(q=None) == C["FA_ERR_INVALID_ARG"]
