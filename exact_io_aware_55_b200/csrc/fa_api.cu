@@ -99,6 +99,21 @@ bool make_map(CUtensorMap* map, const void* base, bool e4m3, int d, int N, int B
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over the backward's fp32 dQ accumulator [BH, N, d]: dims
+// {d, N, BH}, box {32 columns (128 bytes), 128 rows, 1 head}, 128-byte swizzle.
+bool make_map_dq(CUtensorMap* map, void* base, int d, int N, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(N) * d * 4};
+  cuuint32_t box[3] = {32u, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Tensor map over the standard path's probabilities P [BH, N, Np] bf16:
 // dims {Np, N, BH}, box {64 columns, 128 rows, 1 head}, 128-byte swizzle.
 bool make_map_p(CUtensorMap* map, const void* base, int Np, int N, int BH) {
@@ -327,8 +342,10 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   a.BH = BH;
   a.c_log2 = scale * kLog2e;
   a.scale = scale;
+  CUtensorMap tdq;
+  if (!make_map_dq(&tdq, a.dq_acc, d, N, BH)) return FA_ERR_LAUNCH;
   return launch_status(
-      fa::launch_bwd(tq, tk, tv, tdo, a, d, causal != 0, deterministic, static_cast<cudaStream_t>(stream)));
+      fa::launch_bwd(tq, tk, tv, tdo, tdq, a, d, causal != 0, deterministic, static_cast<cudaStream_t>(stream)));
 }
 }  // namespace
 

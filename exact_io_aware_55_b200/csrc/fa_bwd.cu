@@ -22,16 +22,21 @@
 //                  dV_j += P^T dO_i     (A = P^T from TMEM)
 //                  dS^T = scale P^T o (dP^T - D_i) -> shared memory (bf16, swizzled)
 //                  dK_j += dS^T Q_i     (A = dS^T, K-major)
-//                  dQ_i^T = K_j^T dS^T  -> TMEM R2 (both operands read MN-major
-//                                          from the K tile and the dS^T bytes),
-//                                          then fp32 red.add into the workspace
-//                                          accumulator, one d-contiguous line per
-//                                          query row
+//                  d = 128: dQ_i^T = K_j^T dS^T -> TMEM R2 (both operands read
+//                           MN-major from the K tile and the dS^T bytes), then
+//                           fp32 red.add into the workspace accumulator, one
+//                           d-contiguous line per query row
+//                  d = 64:  dQ_i = dS K_j -> TMEM R2 (dS read MN-major from the
+//                           dS^T bytes, K MN-major), staged in shared memory and
+//                           added to the accumulator by one TMA bulk reduction
+//                           per 32 columns (shared memory has room for the
+//                           staging tiles only at d = 64)
 //   bwd_dq_final dQ accumulator -> bf16.
 // Warp roles in bwd_kernel: 0 TMA producer, 1 MMA issuer (+TMEM owner),
 // 4-7 and 8-11 the two P / dS warpgroups (thread = key row = TMEM lane; each
 // handles 64 of the 128 queries of a tile), 12-15 the dQ warpgroup (thread =
-// d index of dQ^T).  Epilogue: warps 4-7 store dV, 8-11 dK.
+// d index of dQ^T at d = 128, query row of dQ at d = 64).  Epilogue: warps 4-7
+// store dV, 8-11 dK.
 // TMEM columns: dV [0,d) dK [d,2d) R1 [2d,2d+128) R2 [2d+128,2d+256).
 #include <cuda_bf16.h>
 
@@ -124,6 +129,12 @@ struct BwdShape {
   // dQ^T = K^T dS^T: M = d (key-tile rows become TMEM lanes = d), N = 128
   // queries, both operands MN-major (the K tile and the dS^T buffer as stored).
   static constexpr uint32_t kIdDQT = idesc_bf16(D, 128, true, true);
+  // d = 64: dQ = dS K: M = 128 queries, N = d; A = dS^T bytes read MN-major,
+  // B = K tile MN-major.  The fp32 tile is staged (two buffers of 128 rows x
+  // 256 bytes, 128-byte swizzled 32-column chunks) for TMA bulk reductions.
+  static constexpr bool kTmaDQ = (D == 64);
+  static constexpr uint32_t kIdDQ = idesc_bf16(128, D, true, true);
+  static constexpr int kStageDQBytes = kTmaDQ ? 128 * D * 4 : 0;
   static constexpr uint32_t kColDV = 0, kColDK = D, kColR1 = 2 * D, kColR2 = 2 * D + 128;
   // Exponentials per 8 pairs computed on the FMA pipe on fully unmasked tiles.
   static constexpr int kEmuPer8 = (D == 64) ? 3 : 2;
@@ -135,6 +146,7 @@ struct BwdBarriers {
   uint64_t qdo_full[NST];
   uint64_t qdo_empty[NST];
   uint64_t s_ready, dp_ready, p_ready, ds_ready, ds_free, dq_ready, dq_free, final_;
+  uint64_t dq_staged[2], dq_stage_free[2];   // TMA-reduced dQ (d = 64)
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -142,7 +154,8 @@ struct BwdBarriers {
 template <int D>
 constexpr size_t bwd_smem_bytes() {
   using S = BwdShape<D>;
-  return size_t(2 + 2 * S::kNST) * S::kTileBytes + S::kDsBytes + S::kNST * 1024 + sizeof(BwdBarriers<S::kNST>);
+  return size_t(2 + 2 * S::kNST) * S::kTileBytes + S::kDsBytes + 2 * size_t(S::kStageDQBytes) + S::kNST * 1024 +
+         sizeof(BwdBarriers<S::kNST>);
 }
 
 __device__ __forceinline__ void red_add_f32(float* addr, float a) {
@@ -159,12 +172,12 @@ template <int D, bool CAUSAL, bool DQ>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-               const BwdArgs args) {
+               const __grid_constant__ CUtensorMap tmdQacc, const BwdArgs args) {
   using S = BwdShape<D>;
   constexpr int NST = S::kNST;
   extern __shared__ __align__(1024) uint8_t smem[];
-  auto* bars =
-      reinterpret_cast<BwdBarriers<NST>*>(smem + (2 + 2 * NST) * S::kTileBytes + S::kDsBytes + NST * 1024);
+  auto* bars = reinterpret_cast<BwdBarriers<NST>*>(smem + (2 + 2 * NST) * S::kTileBytes + S::kDsBytes +
+                                                    2 * S::kStageDQBytes + NST * 1024);
   // The layout relies on a 1024-byte aligned dynamic shared-memory base (the
   // 128-byte swizzle atoms); refuse to run otherwise.
   if ((smem_u32(smem) & 1023u) != 0u) {
@@ -179,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = sV + S::kTileBytes;                 // NST tiles
   uint8_t* sdO = sQ + NST * S::kTileBytes;          // NST tiles
   uint8_t* sdS = sdO + NST * S::kTileBytes;         // dS^T: rows = keys, 128 queries each
-  float* sStat = reinterpret_cast<float*>(sdS + S::kDsBytes);     // per stage: lse2[128], D[128]
+  uint8_t* sdQ = sdS + S::kDsBytes;                 // d = 64: two fp32 dQ staging tiles
+  float* sStat = reinterpret_cast<float*>(sdQ + 2 * S::kStageDQBytes);   // per stage: lse2[128], D[128]
   const WaitCtx wc{&bars->abort, args.status, FA_WAIT_LIMIT_NS};
 
   const int warp = threadIdx.x >> 5;
@@ -207,6 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->dq_ready, 1);
     mbar_init(&bars->dq_free, 4);
     mbar_init(&bars->final_, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->dq_staged[b], 4);
+      mbar_init(&bars->dq_stage_free[b], 1);
+    }
     bars->abort = 0u;
     fence_mbar_init();
   }
@@ -320,7 +338,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dQ^T = K^T dS^T: A = K read MN-major (M = d), B = the dS^T bytes read
         // MN-major (N = queries); 16 keys per step.  The transposed product puts
         // d on the TMEM lanes, so each dQ row update is one coalesced line.
-        if constexpr (DQ) {
+        if constexpr (DQ && S::kTmaDQ) {
+          // dQ = dS K: A = the dS^T bytes read MN-major (M = queries), B = K MN-major (N = d).
+#pragma unroll
+          for (int kt = 0; kt < 8; ++kt)
+            mma_f16_ss_e(tR2, ddS_mn + uint64_t(kt * 128), dK_mn + uint64_t(kt * 128), S::kIdDQ, kt > 0 ? 1u : 0u);
+          tc_commit_e(&bars->dq_ready);
+        } else if constexpr (DQ) {
 #pragma unroll
           for (int kt = 0; kt < 8; ++kt)
             mma_f16_ss_e(tR2, dK_mn + uint64_t(kt * 128), ddS_mn + uint64_t(kt * 128), S::kIdDQT, kt > 0 ? 1u : 0u);
@@ -445,6 +469,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+  } else if (DQ && S::kTmaDQ) {
+    regs_inc<kRegsDQ>();
+    // ------------------------------------------- dQ group, TMA reduction
+    // Thread = query row of the dQ tile in TMEM R2 (lane = row, columns = d).
+    // Per query tile: load the row, write it into staging buffer it % 2
+    // (two 32-column chunks of 128-byte swizzled rows, the layout of the
+    // accumulator's tensor map), and lane 0 of warp 12 adds both chunks to the
+    // accumulator with TMA bulk reductions.  A staging buffer is reused once
+    // the reduction that read it two tiles earlier has finished reading.
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
+    const bool issuer = (warp == 12);
+    bool ok = true;
+    for (int it = 0; it < n_iter && ok; ++it) {
+      const int i = i_begin + it;
+      const int b = it & 1;
+      if (!mbar_wait_warp(&bars->dq_ready, it & 1, wc, WAIT_BWD_DQ)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld_x64(lane_base + S::kColR2, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->dq_free);
+      if (it >= 2 && !mbar_wait_warp(&bars->dq_stage_free[b], ((it >> 1) + 1) & 1, wc, WAIT_BWD_DQ_FREE)) {
+        ok = false;
+        break;
+      }
+      uint8_t* row = sdQ + b * S::kStageDQBytes + r * 128;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(row + c * 16384 + ((u ^ (r & 7)) << 4)) =
+              make_uint4(v[32 * c + 4 * u], v[32 * c + 4 * u + 1], v[32 * c + 4 * u + 2], v[32 * c + 4 * u + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->dq_staged[b]);
+      if (issuer) {
+        if (!mbar_wait_warp(&bars->dq_staged[b], (it >> 1) & 1, wc, WAIT_BWD_DQ)) { ok = false; break; }
+        if (lane == 0) {
+          tma_reduce_add_3d(&tmdQacc, sdQ + b * S::kStageDQBytes, 0, i * kTile, bh);
+          tma_reduce_add_3d(&tmdQacc, sdQ + b * S::kStageDQBytes + 16384, 32, i * kTile, bh);
+          bulk_commit_group();
+          bulk_wait_group_read<1>();                  // the reduction of tile it - 1 has read its buffer
+          if (it >= 1) mbar_arrive(&bars->dq_stage_free[b ^ 1]);
+        }
+        __syncwarp();
+      }
+    }
+    if (issuer && lane == 0) bulk_wait_group<0>();    // every reduction complete before the CTA ends
   } else if (DQ) {
     regs_inc<kRegsDQ>();
     // ---------------------------------------------------------- dQ group
@@ -487,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool CAUSAL, bool DQ>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const BwdArgs& a, cudaStream_t stream) {
+                         const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream) {
   // 1) preprocess + zero the dQ accumulator
   constexpr int RPB = 256 / (D / 8);
   const long long rows = (long long)a.BH * a.Np;
@@ -503,7 +578,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((a.N + kTile - 1) / kTile, a.BH);
-  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, a);
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tdq, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if constexpr (!DQ) {
@@ -520,17 +595,18 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 }  // namespace
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                       const BwdArgs& a, int d, bool causal, bool deterministic, cudaStream_t stream) {
+                       const CUtensorMap& tdq, const BwdArgs& a, int d, bool causal, bool deterministic,
+                       cudaStream_t stream) {
   if (deterministic) {
-    if (d == 64) return causal ? launch_bwd_t<64, true, false>(tq, tk, tv, tdo, a, stream)
-                               : launch_bwd_t<64, false, false>(tq, tk, tv, tdo, a, stream);
-    return causal ? launch_bwd_t<128, true, false>(tq, tk, tv, tdo, a, stream)
-                  : launch_bwd_t<128, false, false>(tq, tk, tv, tdo, a, stream);
+    if (d == 64) return causal ? launch_bwd_t<64, true, false>(tq, tk, tv, tdo, tdq, a, stream)
+                               : launch_bwd_t<64, false, false>(tq, tk, tv, tdo, tdq, a, stream);
+    return causal ? launch_bwd_t<128, true, false>(tq, tk, tv, tdo, tdq, a, stream)
+                  : launch_bwd_t<128, false, false>(tq, tk, tv, tdo, tdq, a, stream);
   }
-  if (d == 64) return causal ? launch_bwd_t<64, true, true>(tq, tk, tv, tdo, a, stream)
-                             : launch_bwd_t<64, false, true>(tq, tk, tv, tdo, a, stream);
-  return causal ? launch_bwd_t<128, true, true>(tq, tk, tv, tdo, a, stream)
-                : launch_bwd_t<128, false, true>(tq, tk, tv, tdo, a, stream);
+  if (d == 64) return causal ? launch_bwd_t<64, true, true>(tq, tk, tv, tdo, tdq, a, stream)
+                             : launch_bwd_t<64, false, true>(tq, tk, tv, tdo, tdq, a, stream);
+  return causal ? launch_bwd_t<128, true, true>(tq, tk, tv, tdo, tdq, a, stream)
+                : launch_bwd_t<128, false, true>(tq, tk, tv, tdo, tdq, a, stream);
 }
 
 }  // namespace fa

@@ -331,12 +331,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       float sv[128];
+      {
+        uint32_t r[128];
+        tmem_ld_x128(s_tmem, r);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t r[32];
-        tmem_ld_x32(s_tmem + q * 32, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[q * 32 + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 128; ++i) sv[i] = __uint_as_float(r[i]);
       }
       const int k0 = j * kBN;
       const bool need_mask = (k0 + kBN > N) || (CAUSAL && k0 + kBN - 1 > q0g);

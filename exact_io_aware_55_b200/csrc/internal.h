@@ -128,9 +128,11 @@ cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const FwdArgs& a, int d, bool causal, cudaStream_t stream);
 cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdArgs& a, int d, bool causal, cudaStream_t stream);
+// tdq: map over the fp32 dQ accumulator (dims {d, N, BH}, box {32 columns,
+// 128 rows}); used by the d = 64 kernel's TMA bulk reductions.
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const BwdArgs& a, int d, bool causal, bool deterministic,
-                       cudaStream_t stream);
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int d, bool causal,
+                       bool deterministic, cudaStream_t stream);
 // Deterministic dQ pass (one 128-query tile per CTA, no atomics); defined in
 // fa_bwd_dq.cu, launched by launch_bwd after the dK/dV kernel.
 template <int D, bool CAUSAL>
