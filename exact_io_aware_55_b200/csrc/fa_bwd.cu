@@ -135,9 +135,15 @@ struct BwdShape {
   static constexpr bool kTmaDQ = (D == 64);
   static constexpr uint32_t kIdDQ = idesc_bf16(128, D, true, true);
   static constexpr int kStageDQBytes = kTmaDQ ? 128 * D * 4 : 0;
+  // d = 64 leaves TMEM columns [384, 512) free: dQ gets its own region there,
+  // so the next dP^T does not wait for the dQ warpgroup to read dQ out.
+  static constexpr uint32_t kColDQ = kTmaDQ ? 384u : uint32_t(2 * D + 128);
   static constexpr uint32_t kColDV = 0, kColDK = D, kColR1 = 2 * D, kColR2 = 2 * D + 128;
   // Exponentials per 8 pairs computed on the FMA pipe on fully unmasked tiles.
-  static constexpr int kEmuPer8 = (D == 64) ? 3 : 2;
+  // None: measured on B200, moving 2/8 or 3/8 of them off MUFU made this
+  // kernel slower (12-20 % at d = 64), the extra FMA-pipe instructions cost
+  // more issue slots than the MUFU unit saves here.
+  static constexpr int kEmuPer8 = 0;
 };
 
 template <int NST>
@@ -305,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < n_iter; ++it) {
         const int s = it % NST;
         const uint64_t st = uint64_t(s) * kTileD;
-        if (DQ && it > 0) {
+        if (DQ && !S::kTmaDQ && it > 0) {       // dP^T reuses R2, where dQ^T was
           if (!mbar_wait_warp(&bars->dq_free, (it - 1) & 1, wc, WAIT_BWD_DQ_FREE)) { ok = false; break; }
           tc_fence_after();
         }
@@ -339,10 +345,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // MN-major (N = queries); 16 keys per step.  The transposed product puts
         // d on the TMEM lanes, so each dQ row update is one coalesced line.
         if constexpr (DQ && S::kTmaDQ) {
-          // dQ = dS K: A = the dS^T bytes read MN-major (M = queries), B = K MN-major (N = d).
+          // dQ = dS K: A = the dS^T bytes read MN-major (M = queries), B = K MN-major (N = d),
+          // into its own TMEM region once the dQ warpgroup has read the previous tile.
+          if (it > 0) {
+            if (!mbar_wait_warp(&bars->dq_free, (it - 1) & 1, wc, WAIT_BWD_DQ_FREE)) { ok = false; break; }
+            tc_fence_after();
+          }
 #pragma unroll
           for (int kt = 0; kt < 8; ++kt)
-            mma_f16_ss_e(tR2, ddS_mn + uint64_t(kt * 128), dK_mn + uint64_t(kt * 128), S::kIdDQ, kt > 0 ? 1u : 0u);
+            mma_f16_ss_e(tmem + S::kColDQ, ddS_mn + uint64_t(kt * 128), dK_mn + uint64_t(kt * 128), S::kIdDQ,
+                         kt > 0 ? 1u : 0u);
           tc_commit_e(&bars->dq_ready);
         } else if constexpr (DQ) {
 #pragma unroll
@@ -489,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_warp(&bars->dq_ready, it & 1, wc, WAIT_BWD_DQ)) { ok = false; break; }
       tc_fence_after();
       uint32_t v[64];
-      tmem_ld_x64(lane_base + S::kColR2, v);
+      tmem_ld_x64(lane_base + S::kColDQ, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->dq_free);
