@@ -101,16 +101,16 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a, int row_blocks,
 
 // ------------------------------------------------------------ dQ finalize
 __global__ void __launch_bounds__(256) bwd_dq_final_kernel(const float* __restrict__ acc, __nv_bfloat16* dq,
-                                                           long long n8) {
+                                                           long long n8, float scale) {
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n8; t += stride) {
     const float4 x = reinterpret_cast<const float4*>(acc)[2 * t];
     const float4 y = reinterpret_cast<const float4*>(acc)[2 * t + 1];
     uint4 o;
-    o.x = pack_bf16x2(x.x, x.y);
-    o.y = pack_bf16x2(x.z, x.w);
-    o.z = pack_bf16x2(y.x, y.y);
-    o.w = pack_bf16x2(y.z, y.w);
+    o.x = pack_bf16x2(x.x * scale, x.y * scale);
+    o.y = pack_bf16x2(x.z * scale, x.w * scale);
+    o.z = pack_bf16x2(y.x * scale, y.y * scale);
+    o.w = pack_bf16x2(y.z * scale, y.w * scale);
     reinterpret_cast<uint4*>(dq)[t] = o;
   }
 }
@@ -135,6 +135,7 @@ struct BwdShape {
   static constexpr bool kTmaDQ = (D == 64);
   static constexpr uint32_t kIdDQ = idesc_bf16(128, D, true, true);
   static constexpr int kStageDQBytes = kTmaDQ ? 128 * D * 4 : 0;
+  static_assert(kIdDQ != 0 && kIdDQT != 0, "both dQ forms are defined for every d");
   // d = 64 leaves TMEM columns [384, 512) free: dQ gets its own region there,
   // so the next dP^T does not wait for the dQ warpgroup to read dQ out.
   static constexpr uint32_t kColDQ = kTmaDQ ? 384u : uint32_t(2 * D + 128);
@@ -382,7 +383,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tP = lane_base + S::kColR1 + 96 * h;        // its P^T (bf16) columns
     const uint32_t tdP = lane_base + S::kColR2 + 64 * h;       // this half's dP^T columns
     const float cl = args.c_log2;
-    const float scale = args.scale;
     const bool kv_valid = kv < N;
     const bool kv_tile_full = (j + 1) * kTile <= N;
     uint8_t* ds_row = sdS + h * 16384 + (c >> 3) * 1024 + (c & 7) * 128;
@@ -406,7 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 cc = make_float2(cl, cl);
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const float2 nl = *reinterpret_cast<const float2*>(snl + 2 * t);
+          const float4 nl4 = *reinterpret_cast<const float4*>(snl + 4 * (t >> 1));
+          const float2 nl = (t & 1) ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
           const float2 x = ffma2(make_float2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1])), cc, nl);
           float2 p;
           if (!exact && (t & 7) < S::kEmuPer8) {
@@ -428,21 +429,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);
-      // dS^T row = scale * P^T o (dP^T - D_q) -> shared memory, 128-byte swizzled K-major rows.
+      // dS^T row = P^T o (dP^T - D_q) -> shared memory, 128-byte swizzled K-major rows.  The
+      // factor scale of dS is applied once to dK (epilogue) and dQ (finalize) instead.
       if (!mbar_wait_warp(&bars->dp_ready, it & 1, wc, WAIT_BWD_DP)) { ok = false; break; }
       if (it > 0 && !mbar_wait_warp(&bars->ds_free, (it - 1) & 1, wc, WAIT_BWD_DS_FREE)) { ok = false; break; }
       tc_fence_after();
       {
         uint32_t r[64];
         tmem_ld_x64(tdP, r);
-        const float2 sc2 = make_float2(scale, scale);
         uint32_t w[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const float2 nd = *reinterpret_cast<const float2*>(snd + 2 * t);
+          const float4 nd4 = *reinterpret_cast<const float4*>(snd + 4 * (t >> 1));
+          const float2 nd = (t & 1) ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
           const float2 dpm = fadd2(make_float2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1])), nd);
-          const float2 ps = fmul2(make_float2(bf16lo(pk[t]), bf16hi(pk[t])), sc2);
-          const float2 ds = fmul2(ps, dpm);
+          const float2 ds = fmul2(make_float2(bf16lo(pk[t]), bf16hi(pk[t])), dpm);
           w[t] = pack_bf16x2(ds.x, ds.y);
         }
         // 64 queries = 128 bytes = one full row of chunk h, eight 16-byte units.
@@ -464,6 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(h == 0 ? args.dv : args.dk) + (size_t(bh) * N + kv) * D;
       const uint32_t src = lane_base + (h == 0 ? S::kColDV : S::kColDK);
+      const float f = (h == 0) ? 1.0f : args.scale;   // dK = scale * dS^T Q
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         uint32_t r[32];
@@ -472,10 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]), __uint_as_float(r[8 * u + 1]));
-            v.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]), __uint_as_float(r[8 * u + 3]));
-            v.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]), __uint_as_float(r[8 * u + 5]));
-            v.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]), __uint_as_float(r[8 * u + 7]));
+            v.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * f, __uint_as_float(r[8 * u + 1]) * f);
+            v.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * f, __uint_as_float(r[8 * u + 3]) * f);
+            v.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * f, __uint_as_float(r[8 * u + 5]) * f);
+            v.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * f, __uint_as_float(r[8 * u + 7]) * f);
             reinterpret_cast<uint4*>(dst + q * 32)[u] = v;
           }
         }
@@ -600,7 +602,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   // 3) dQ -> bf16
   const long long n8 = (long long)a.BH * a.N * D / 8;
   const int fin_blocks = int(std::min<long long>((n8 + 255) / 256, 148LL * 8));
-  bwd_dq_final_kernel<<<fin_blocks, 256, 0, stream>>>(a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq), n8);
+  bwd_dq_final_kernel<<<fin_blocks, 256, 0, stream>>>(a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq), n8, a.scale);
   return cudaGetLastError();
 }
 
