@@ -161,6 +161,21 @@ WsLayout ws_layout(long long BH, int N, int d) {
   return w;
 }
 
+// Heads per ordering group of the causal grids: as many as keep the group's
+// streamed operands (K/V in the forward; Q, dO and the fp32 dQ rows in the
+// backward) within 64 MiB of L2.
+int head_group(long long bytes_per_head, int BH) {
+  const long long budget = 64ll << 20;
+  long long g = bytes_per_head > 0 ? budget / bytes_per_head : BH;
+  if (g < 1) g = 1;
+  if (g > BH) g = BH;
+  return static_cast<int>(g);
+}
+
+// Causal grids are 1-D with BH * ceil(N / 128) blocks (an upper bound for
+// every kernel's unit count); that must fit in a signed 32-bit index.
+bool causal_grid_fits(long long BH, int N) { return BH * ((static_cast<long long>(N) + 127) / 128) <= 0x7fffffffll; }
+
 fa_status launch_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH; }
 
 // Split-KV decode plan.  A head's cache is cut into items of whole key tiles
@@ -238,6 +253,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   if (e4m3 && !(std::isfinite(qd) && std::isfinite(kd) && std::isfinite(vd) && qd > 0 && kd > 0 && vd > 0))
     return FA_ERR_INVALID_ARG;
   if (empty) return FA_OK;
+  if (causal && !causal_grid_fits(static_cast<long long>(B) * H, N)) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGNMENT;
@@ -255,6 +271,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   a.BH = BH;
   a.c_log2 = scale * kLog2e * (e4m3 ? qd * kd : 1.0f);
   a.o_scale = e4m3 ? vd : 1.0f;
+  a.head_group = head_group(2ll * N * d * (e4m3 ? 1 : 2), BH);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return launch_status(e4m3 ? fa::launch_fwd_e4m3(tq, tk, tv, a, d, causal != 0, s)
                             : fa::launch_fwd_bf16(tq, tk, tv, a, d, causal != 0, s));
@@ -312,6 +329,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   fa_status st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK) return st;
   if (empty) return FA_OK;
+  if (causal && !causal_grid_fits(static_cast<long long>(B) * H, N)) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   const int BH = B * H;
   const WsLayout wl = ws_layout(BH, N, d);
@@ -342,6 +360,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   a.BH = BH;
   a.c_log2 = scale * kLog2e;
   a.scale = scale;
+  a.head_group = head_group(8ll * N * d, BH);   // Q, dO (bf16) and the fp32 dQ rows of a head
   CUtensorMap tdq;
   if (!make_map_dq(&tdq, a.dq_acc, d, N, BH)) return FA_ERR_LAUNCH;
   return launch_status(

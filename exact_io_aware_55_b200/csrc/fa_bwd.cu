@@ -207,10 +207,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   // Grid: x = key tile (fastest), y = batch-head, so the CTAs resident at any
   // time cover few heads: their Q/dO tiles and dQ accumulator rows stay in L2.
-  const int bh = blockIdx.y;
-  const int j = blockIdx.x;                          // key tile (0 = heaviest when causal)
+  // Causal: a 1-D grid, the heaviest key tiles (the first ones) first across
+  // each group of heads.
   const int N = args.N;
   const int n_q = (N + kTile - 1) / kTile;
+  int bh, j;                                         // key tile j (0 = heaviest when causal)
+  if constexpr (CAUSAL) {
+    causal_block_order(int(blockIdx.x), n_q, args.BH, args.head_group, j, bh);
+  } else {
+    bh = blockIdx.y;
+    j = blockIdx.x;
+  }
   const int i_begin = CAUSAL ? j : 0;
   const int n_iter = n_q - i_begin;
 
@@ -591,7 +598,8 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   auto kern = bwd_kernel<D, CAUSAL, DQ>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.N + kTile - 1) / kTile, a.BH);
+  const int n_t = (a.N + kTile - 1) / kTile;
+  const dim3 grid = CAUSAL ? dim3(unsigned(n_t) * unsigned(a.BH)) : dim3(n_t, a.BH);
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tdq, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -75,9 +75,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int N = args.N;
   const int n_kv = (N + kTile - 1) / kTile;
-  // Grid: x = query tile (fastest; heaviest first when causal), y = batch-head.
-  const int i = CAUSAL ? int(gridDim.x - 1 - blockIdx.x) : int(blockIdx.x);
-  const int bh = blockIdx.y;
+  // Grid: x = query tile (fastest), y = batch-head; causal: a 1-D grid, the
+  // heaviest query tiles (the last ones) first across each group of heads.
+  int i, bh;                                           // query tile i (the last = heaviest when causal)
+  if constexpr (CAUSAL) {
+    int rank;
+    causal_block_order(int(blockIdx.x), int((args.N + kTile - 1) / kTile), args.BH, args.head_group, rank, bh);
+    i = (args.N + kTile - 1) / kTile - 1 - rank;
+  } else {
+    i = blockIdx.x;
+    bh = blockIdx.y;
+  }
   const int T = CAUSAL ? min(n_kv, i + 1) : n_kv;
 
   if (threadIdx.x == 0) {
@@ -293,7 +301,8 @@ cudaError_t launch_bwd_dq(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   auto kern = bwd_dq_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.N + kTile - 1) / kTile, a.BH);
+  const int n_t = (a.N + kTile - 1) / kTile;
+  const dim3 grid = CAUSAL ? dim3(unsigned(n_t) * unsigned(a.BH)) : dim3(n_t, a.BH);
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, a);
   return cudaGetLastError();
 }

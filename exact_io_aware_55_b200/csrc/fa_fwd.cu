@@ -151,11 +151,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   // Grid: x = Q-tile pair (fastest), y = batch-head, so the CTAs resident at
   // any time cover few heads and their K/V tiles are re-read from L2, not HBM.
-  // Causal: heaviest pairs of each head first.
-  const int bh = blockIdx.y;
-  const int pair = CAUSAL ? int(gridDim.x - 1 - blockIdx.x) : int(blockIdx.x);
+  // Causal: a 1-D grid, heaviest pairs (the last ones) first across each group
+  // of heads.
   const int N = args.N;
   const int n_kv = (N + kBN - 1) / kBN;
+  int bh, pair;
+  if constexpr (CAUSAL) {
+    const int n_pairs = (N + kNQT * kBM - 1) / (kNQT * kBM);
+    int rank;
+    causal_block_order(int(blockIdx.x), n_pairs, args.BH, args.head_group, rank, bh);
+    pair = n_pairs - 1 - rank;
+  } else {
+    bh = blockIdx.y;
+    pair = blockIdx.x;
+  }
 
   int q0[kNQT], T[kNQT];
   int Tmax = 0;
@@ -426,7 +435,8 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   auto kern = fwd_kernel<D, CAUSAL, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.N + kNQT * kBM - 1) / (kNQT * kBM), a.BH);
+  const int n_pairs = (a.N + kNQT * kBM - 1) / (kNQT * kBM);
+  const dim3 grid = CAUSAL ? dim3(unsigned(n_pairs) * unsigned(a.BH)) : dim3(n_pairs, a.BH);
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }

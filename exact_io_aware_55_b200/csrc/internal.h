@@ -67,6 +67,7 @@ struct FwdArgs {
   int BH;
   float c_log2;   // scale * log2(e), times the q/k descales for e4m3 inputs
   float o_scale;  // factor applied with 1/l to O (1, or the v descale for e4m3)
+  int head_group; // causal: heads per ordering group (see causal_block_order)
 };
 
 struct BwdArgs {
@@ -85,7 +86,25 @@ struct BwdArgs {
   int BH;
   float c_log2;       // scale * log2(e)
   float scale;
+  int head_group;     // causal: heads per ordering group (see causal_block_order)
 };
+
+// Causal grids are one-dimensional: n_units work units (query-tile pairs,
+// key tiles, query tiles) per head, whose cost grows or shrinks linearly with
+// the unit.  Block b is mapped to (rank, head) so that, within each group of
+// `group` heads, every head's heaviest unit (rank 0) is dispatched first, then
+// every head's next one, and so on; groups follow one another.  The light
+// units fill the SMs at the end of the grid instead of the heaviest units of
+// the last head, and a group's K/V (or Q/dO) stays within an L2-sized budget.
+__device__ __forceinline__ void causal_block_order(int b, int n_units, int BH, int group, int& rank, int& head) {
+  const int per_group = group * n_units;
+  const int g = b / per_group;
+  const int r = b - g * per_group;
+  const int h0 = g * group;
+  const int gsize = min(group, BH - h0);
+  rank = r / gsize;
+  head = h0 + (r - rank * gsize);
+}
 
 struct DecodeArgs {
   uint32_t* status;   // device status words (code, where)
