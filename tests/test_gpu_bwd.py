@@ -117,6 +117,13 @@ def test_bwd_config_b1_h32_n32768_d128_causal_sampled():
     _sampled(1, 32, 32768, 128, True, seed=1238, n_heads=1, n_rows=12)
 
 
+def test_bwd_causal_partial_head_group_b2_h5_n16384_d128_sampled():
+    """Ten heads at N=16384, d=128: the causal grid orders heads in groups of
+    four (Q, dO and the fp32 dQ rows of a head are 16 MiB against a 64 MiB
+    budget), so the last group holds two heads."""
+    _sampled(2, 5, 16384, 128, True, seed=1240, n_heads=3, n_rows=12)
+
+
 def test_bwd_workspace_checks():
     x = torch.zeros((1, 1, 64, 64), dtype=torch.bfloat16, device="cuda")
     lse = torch.zeros((1, 1, 64), dtype=torch.float32, device="cuda")

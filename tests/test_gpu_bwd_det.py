@@ -65,3 +65,13 @@ def test_det_config_b2_h16_n8192_d128_causal_sampled():
         qh, kh, vh, doh = (synth.head_f64(inp, n, b, h) for n in ("q", "k", "v", "do"))
         rq, _, _ = oracle.head_backward_sampled(qh, kh, vh, doh, scale, True, rows, rows[:2])
         assert gu.rel_fro(dq[b, h][rows], rq) <= gu.GRAD_REL_FRO
+
+
+def test_det_matches_atomic_partial_head_group_b2_h5_n16384_d128_causal():
+    """Ten heads at N=16384: both causal grids order heads in groups of four,
+    the last group holding two; the atomic-free dQ pass and the atomic one agree."""
+    inp = synth.attention_inputs(2, 5, 16384, 128, seed=412, want_f64=False)
+    outs, scale, (q, k, v, o, do, lse) = _run(inp, True)
+    ref = fa.attention_backward(q, k, v, o, do, lse, scale=scale, causal=True)
+    for g, r in zip(outs[0], ref):
+        assert gu.rel_fro(gu.to_f64(g), gu.to_f64(r)) <= 5e-3

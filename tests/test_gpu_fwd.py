@@ -93,6 +93,12 @@ def test_fwd_config_b1_h32_n32768_d128_causal_sampled():
     _sampled_check(1, 32, 32768, 128, True, seed=1238, n_heads=2, n_rows=16)
 
 
+def test_fwd_causal_partial_head_group_b2_h5_n16384_d128_sampled():
+    """Ten heads at N=16384, d=128: K and V of a head are 8 MiB, so the causal
+    grid orders heads in groups of eight and the last group holds two."""
+    _sampled_check(2, 5, 16384, 128, True, seed=1240, n_heads=3, n_rows=16)
+
+
 def test_fwd_noncausal_n8192_d128_sampled():
     _sampled_check(1, 32, 8192, 128, False, seed=1239, n_heads=2)
 
