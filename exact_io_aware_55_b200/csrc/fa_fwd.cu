@@ -60,7 +60,7 @@ struct FwdShape {
   // Exponentials per 8 on the FMA pipe (exp2_fma2) instead of MUFU, on tiles
   // without masked entries: where the MMA time per tile is shorter (d = 64,
   // e4m3) the MUFU unit alone would bound the kernel, so more is moved.
-  static constexpr int kEmuPer8 = (D == 64 || FP8) ? 3 : 1;
+  static constexpr int kEmuPer8 = (D == 64 || FP8) ? 3 : 2;
   static constexpr uint32_t kIdS = FP8 ? idesc_e4m3(128, 128, false, false) : idesc_bf16(128, 128, false, false);
   static constexpr uint32_t kIdPV = FP8 ? idesc_e4m3(128, D, false, true) : idesc_bf16(128, D, false, true);
   static_assert(kRowBytes % 128 == 0, "head row must be a whole number of 128-byte chunks");
