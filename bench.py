@@ -390,7 +390,8 @@ def committed_traffic(kernel: str, workload: str):
 
 def extra_measurements(fa, torch, synth, dev, stream):
     """Single-GPU context numbers: long-sequence non-causal bf16 (fwd and bwd at
-    N=8192, d=128), the e4m3 forward at B2 H16 N16384 d128, standard
+    N=8192, d=128), the causal B2 H16 N8192 and B1 H32 N32768 d128
+    configurations, the e4m3 forward at B2 H16 N16384 d128, standard
     (materialising) attention against the fused forward, and the split-KV
     decode (1 and 4 queries over a 16384-key cache, 8 x 32 heads, d=128)."""
     out = {}
@@ -426,6 +427,25 @@ def extra_measurements(fa, torch, synth, dev, stream):
         "bwd_tflops": round(2.5 * F / tb / 1e9, 1), "bwd_frac": round(2.5 * F / tb / 1e9 / peaks["bf16_tflops"], 4),
         "inputs": "N(0,1) from torch's seeded CUDA generator (timing only)"}
     del q, k, v, do, o, dq, dk, dv, work
+    # the named causal configurations: B2 H16 N8192 d128 and B1 H32 N32768 d128
+    for (B, H, N, d) in ((2, 16, 8192, 128), (1, 32, 32768, 128)):
+        q, k, v, do = (torch.randn((B, H, N, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+                       for _ in range(4))
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        work = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+        sc = 1.0 / math.sqrt(d)
+        F = fwd_flops(B, H, N, d, True)
+        it = 10 if N <= 8192 else 4
+        tf = time_call(lambda: fa.fa_fwd(q, k, v, o, lse, sc, True, stream), iters=it)
+        tb = time_call(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, sc, True, work, stream), iters=it)
+        out[f"causal_b{B}_h{H}_n{N}_d{d}"] = {
+            "fwd_tflops": round(F / tf / 1e9, 1), "fwd_frac": round(F / tf / 1e9 / peaks["bf16_tflops"], 4),
+            "bwd_tflops": round(2.5 * F / tb / 1e9, 1),
+            "bwd_frac": round(2.5 * F / tb / 1e9 / peaks["bf16_tflops"], 4),
+            "fwd_bwd_tflops": round(3.5 * F / (tf + tb) / 1e9, 1)}
+        del q, k, v, do, o, dq, dk, dv, work
     B, H, N, d = 2, 16, 16384, 128
     q8, k8, v8 = (torch.randn((B, H, N, d), generator=g, device=dev).mul_(100.0).clamp_(-448, 448)
                   .to(torch.float8_e4m3fn) for _ in range(3))
