@@ -37,7 +37,8 @@
 // handles 64 of the 128 queries of a tile), 12-15 the dQ warpgroup (thread =
 // d index of dQ^T at d = 128, query row of dQ at d = 64).  Epilogue: warps 4-7
 // store dV, 8-11 dK.
-// TMEM columns: dV [0,d) dK [d,2d) R1 [2d,2d+128) R2 [2d+128,2d+256).
+// TMEM columns: dV [0,d) dK [d,2d) R1 [2d,2d+128) R2 [2d+128,2d+256); at d = 64
+// the untransposed dQ tile has its own columns [384, 448).
 #include <cuda_bf16.h>
 
 #include "internal.h"
