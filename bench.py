@@ -139,7 +139,8 @@ def run_ours(args):
         import datetime
 
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        # long enough for rank 0's extra measurements while the others wait at the last barrier
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     dev = torch.device("cuda", local)
     B, H, N, d, causal = (WORKLOAD[k] for k in ("B", "H", "N", "d", "causal"))
     scale = 1.0 / math.sqrt(d)
@@ -199,8 +200,15 @@ def run_ours(args):
         return t_fwd, t_bwd, clocks
 
     t_fwd, t_bwd, clocks = timed(args.steps, args.warmup)
-    if any(r in clocks["reasons"] for r in BAD_REASONS):
-        t_fwd, t_bwd, clocks = timed(args.steps, args.warmup)   # re-measure once
+    # Re-measure once if any rank saw a throttle reason; the decision is taken
+    # together so that every rank runs the same collectives.
+    bad = any(r in clocks["reasons"] for r in BAD_REASONS)
+    if dist is not None:
+        flag = torch.tensor([1.0 if bad else 0.0], device=dev)
+        dist.all_reduce(flag, op=dist.ReduceOp.MAX)
+        bad = flag.item() > 0.0
+    if bad:
+        t_fwd, t_bwd, clocks = timed(args.steps, args.warmup)
         clocks["remeasured"] = True
     st, where = fa.fa_device_status(stream)
     if st != 0:
