@@ -172,9 +172,24 @@ int head_group(long long bytes_per_head, int BH) {
   return static_cast<int>(g);
 }
 
-// Causal grids are 1-D with BH * ceil(N / 128) blocks (an upper bound for
-// every kernel's unit count); that must fit in a signed 32-bit index.
-bool causal_grid_fits(long long BH, int N) { return BH * ((static_cast<long long>(N) + 127) / 128) <= 0x7fffffffll; }
+// Causal grids, and the forward's grids, are 1-D with at most
+// BH * ceil(N / 128) blocks; that must fit in a signed 32-bit index.
+bool grid_fits(long long BH, int N) { return BH * ((static_cast<long long>(N) + 127) / 128) <= 0x7fffffffll; }
+
+// Non-causal forward: blocks take Q-tile pairs.  When the pairs leave a last
+// round that fills at most half the SMs, that round's pairs are split into
+// single-tile blocks (twice as many, each about half as long), so the tail
+// runs on up to all SMs.  Only when every pair has two tiles (an even number
+// of 128-row tiles), so that no block is ever empty.
+int sm_count();
+int fwd_pair_blocks(long long BH, int N) {
+  const long long n_qt = (static_cast<long long>(N) + 127) / 128;
+  const long long pairs = BH * ((n_qt + 1) / 2);
+  const long long sms = sm_count();
+  const long long rem = pairs % sms;
+  if (n_qt % 2 != 0 || rem == 0 || 2 * rem > sms) return static_cast<int>(pairs);
+  return static_cast<int>(pairs - rem);
+}
 
 fa_status launch_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH; }
 
@@ -253,7 +268,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   if (e4m3 && !(std::isfinite(qd) && std::isfinite(kd) && std::isfinite(vd) && qd > 0 && kd > 0 && vd > 0))
     return FA_ERR_INVALID_ARG;
   if (empty) return FA_OK;
-  if (causal && !causal_grid_fits(static_cast<long long>(B) * H, N)) return FA_ERR_UNSUPPORTED;
+  if (!grid_fits(static_cast<long long>(B) * H, N)) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGNMENT;
@@ -272,6 +287,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   a.c_log2 = scale * kLog2e * (e4m3 ? qd * kd : 1.0f);
   a.o_scale = e4m3 ? vd : 1.0f;
   a.head_group = head_group(2ll * N * d * (e4m3 ? 1 : 2), BH);
+  a.pair_blocks = fwd_pair_blocks(BH, N);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return launch_status(e4m3 ? fa::launch_fwd_e4m3(tq, tk, tv, a, d, causal != 0, s)
                             : fa::launch_fwd_bf16(tq, tk, tv, a, d, causal != 0, s));
@@ -329,7 +345,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   fa_status st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK) return st;
   if (empty) return FA_OK;
-  if (causal && !causal_grid_fits(static_cast<long long>(B) * H, N)) return FA_ERR_UNSUPPORTED;
+  if (causal && !grid_fits(static_cast<long long>(B) * H, N)) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   const int BH = B * H;
   const WsLayout wl = ws_layout(BH, N, d);

@@ -155,23 +155,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   // of heads.
   const int N = args.N;
   const int n_kv = (N + kBN - 1) / kBN;
-  int bh, pair;
+  // Non-causal: a 1-D grid over (head, pair) in that order, pair fastest.  The
+  // pairs after `pair_blocks` are split, one Q tile per block, so that the last
+  // round of an uneven grid runs short single-tile blocks on many SMs instead
+  // of full pairs on a few.
+  const int n_pairs = (N + kNQT * kBM - 1) / (kNQT * kBM);
+  int bh, pair, only = -1;   // only >= 0: this block takes Q tile `only` of its pair alone
   if constexpr (CAUSAL) {
-    const int n_pairs = (N + kNQT * kBM - 1) / (kNQT * kBM);
     int rank;
     causal_block_order(int(blockIdx.x), n_pairs, args.BH, args.head_group, rank, bh);
     pair = n_pairs - 1 - rank;
   } else {
-    bh = blockIdx.y;
-    pair = blockIdx.x;
+    int p = int(blockIdx.x);
+    if (p >= args.pair_blocks) {
+      const int u = p - args.pair_blocks;
+      p = args.pair_blocks + (u >> 1);
+      only = u & 1;
+    }
+    bh = p / n_pairs;
+    pair = p - bh * n_pairs;
   }
 
   int q0[kNQT], T[kNQT];
   int Tmax = 0;
 #pragma unroll
   for (int g = 0; g < kNQT; ++g) {
-    q0[g] = pair * (kNQT * kBM) + g * kBM;
-    T[g] = (q0[g] < N) ? (CAUSAL ? min(n_kv, q0[g] / kBN + 1) : n_kv) : 0;
+    // a single-tile block runs its tile as Q tile 0; the other slot is empty
+    q0[g] = pair * (kNQT * kBM) + (only >= 0 ? only : g) * kBM;
+    T[g] = (q0[g] < N && (only < 0 || g == 0)) ? (CAUSAL ? min(n_kv, q0[g] / kBN + 1) : n_kv) : 0;
     Tmax = max(Tmax, T[g]);
   }
 
@@ -323,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = (warp - 4) >> 2;
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;
-    const int q0g = pair * (kNQT * kBM) + g * kBM;
-    const int Tg = (q0g < N) ? (CAUSAL ? min(n_kv, q0g / kBN + 1) : n_kv) : 0;
+    const int q0g = pair * (kNQT * kBM) + (only >= 0 ? only : g) * kBM;
+    const int Tg = (q0g < N && (only < 0 || g == 0)) ? (CAUSAL ? min(n_kv, q0g / kBN + 1) : n_kv) : 0;
     const int qrow = q0g + row;
     const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
     const uint32_t s_tmem = lane_base + uint32_t(g * 128);
@@ -435,9 +446,10 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   auto kern = fwd_kernel<D, CAUSAL, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  const int n_pairs = (a.N + kNQT * kBM - 1) / (kNQT * kBM);
-  const dim3 grid = CAUSAL ? dim3(unsigned(n_pairs) * unsigned(a.BH)) : dim3(n_pairs, a.BH);
-  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, a);
+  const unsigned n_pairs = unsigned((a.N + kNQT * kBM - 1) / (kNQT * kBM));
+  const unsigned pairs = n_pairs * unsigned(a.BH);
+  const unsigned blocks = CAUSAL ? pairs : unsigned(a.pair_blocks) + 2u * (pairs - unsigned(a.pair_blocks));
+  kern<<<dim3(blocks), kThreads, smem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

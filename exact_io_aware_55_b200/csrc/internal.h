@@ -68,6 +68,8 @@ struct FwdArgs {
   float c_log2;   // scale * log2(e), times the q/k descales for e4m3 inputs
   float o_scale;  // factor applied with 1/l to O (1, or the v descale for e4m3)
   int head_group; // causal: heads per ordering group (see causal_block_order)
+  int pair_blocks; // non-causal: blocks [0, pair_blocks) take a Q-tile pair each; the
+                   // blocks after them take the two tiles of the following pairs one at a time
 };
 
 struct BwdArgs {
