@@ -288,6 +288,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   a.o_scale = e4m3 ? vd : 1.0f;
   a.head_group = head_group(2ll * N * d * (e4m3 ? 1 : 2), BH);
   a.pair_blocks = fwd_pair_blocks(BH, N);
+  a.max_ctas = sm_count();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return launch_status(e4m3 ? fa::launch_fwd_e4m3(tq, tk, tv, a, d, causal != 0, s)
                             : fa::launch_fwd_bf16(tq, tk, tv, a, d, causal != 0, s));

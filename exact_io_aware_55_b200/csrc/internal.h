@@ -17,6 +17,9 @@ enum WaitSite : uint32_t {
   WAIT_FWD_S = 5,
   WAIT_FWD_P = 6,
   WAIT_FWD_O = 7,
+  WAIT_FWD_S_FREE = 8,
+  WAIT_FWD_PV = 9,
+  WAIT_FWD_Q_EMPTY = 10,
   WAIT_BWD_KV = 16,
   WAIT_BWD_QDO = 17,
   WAIT_BWD_QDO_EMPTY = 18,
@@ -70,6 +73,7 @@ struct FwdArgs {
   int head_group; // causal: heads per ordering group (see causal_block_order)
   int pair_blocks; // non-causal: blocks [0, pair_blocks) take a Q-tile pair each; the
                    // blocks after them take the two tiles of the following pairs one at a time
+  int max_ctas;    // d = 64 non-causal: persistent grid size (the SM count); 0 = one item per CTA
 };
 
 struct BwdArgs {
@@ -149,6 +153,9 @@ cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const FwdArgs& a, int d, bool causal, cudaStream_t stream);
 cudaError_t launch_fwd_e4m3(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdArgs& a, int d, bool causal, cudaStream_t stream);
+// d = 64 bf16 forward (fa_fwd64.cu); launch_fwd_bf16 forwards d = 64 here.
+cudaError_t launch_fwd64(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdArgs& a,
+                         bool causal, cudaStream_t stream);
 // tdq: map over the fp32 dQ accumulator (dims {d, N, BH}, box {32 columns,
 // 128 rows}); used by the d = 64 kernel's TMA bulk reductions.
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
