@@ -170,9 +170,6 @@ __device__ __forceinline__ void red_add_f32(float* addr, float a) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
 }
 
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
 // DQ = false: deterministic mode; this kernel produces dK and dV only and
 // the dQ^T product, its reductions and the dQ warpgroup are skipped (dQ comes
 // from bwd_dq_kernel).
@@ -408,6 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool diag = CAUSAL && (i == j);
       const bool exact = diag || !kv_tile_full || (i + 1) * kTile > N;
       uint32_t pk[32];
+      float2 pf[32];                                  // P in fp32, for dS
       {
         uint32_t r[64];
         tmem_ld_x64(tS, r);
@@ -429,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!kv_valid) p = make_float2(0.0f, 0.0f);
           }
+          pf[t] = p;
           pk[t] = pack_bf16x2(p.x, p.y);
         }
       }
@@ -437,27 +436,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_ready);
-      // dS^T row = P^T o (dP^T - D_q) -> shared memory, 128-byte swizzled K-major rows.  The
-      // factor scale of dS is applied once to dK (epilogue) and dQ (finalize) instead.
+      // dS^T row = P^T o (dP^T - D_q) -> shared memory, 128-byte swizzled K-major rows, from
+      // the fp32 P (its bf16 copy feeds only dV).  The factor scale of dS is applied once
+      // to dK (epilogue) and dQ (finalize) instead.
       if (!mbar_wait_warp(&bars->dp_ready, it & 1, wc, WAIT_BWD_DP)) { ok = false; break; }
       if (it > 0 && !mbar_wait_warp(&bars->ds_free, (it - 1) & 1, wc, WAIT_BWD_DS_FREE)) { ok = false; break; }
       tc_fence_after();
-      {
-        uint32_t r[64];
-        tmem_ld_x64(tdP, r);
-        uint32_t w[32];
+      // 64 queries = 128 bytes = one full row of chunk h, eight 16-byte units;
+      // dP^T in two 32-column pieces.
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
+      for (int q = 0; q < 2; ++q) {
+        uint32_t r[32];
+        tmem_ld_x32(tdP + 32 * q, r);
+        uint32_t w[16];
+#pragma unroll
+        for (int t2 = 0; t2 < 16; ++t2) {
+          const int t = 16 * q + t2;
           const float4 nd4 = *reinterpret_cast<const float4*>(snd + 4 * (t >> 1));
           const float2 nd = (t & 1) ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
-          const float2 dpm = fadd2(make_float2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1])), nd);
-          const float2 ds = fmul2(make_float2(bf16lo(pk[t]), bf16hi(pk[t])), dpm);
-          w[t] = pack_bf16x2(ds.x, ds.y);
+          const float2 dpm = fadd2(make_float2(__uint_as_float(r[2 * t2]), __uint_as_float(r[2 * t2 + 1])), nd);
+          const float2 ds = fmul2(pf[t], dpm);
+          w[t2] = pack_bf16x2(ds.x, ds.y);
         }
-        // 64 queries = 128 bytes = one full row of chunk h, eight 16-byte units.
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<uint4*>(ds_row + ((u ^ (c & 7)) << 4)) =
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(ds_row + (((4 * q + u) ^ (c & 7)) << 4)) =
               make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       }
       fence_proxy_async_smem();
