@@ -38,7 +38,8 @@
 // d index of dQ^T at d = 128, query row of dQ at d = 64).  Epilogue: warps 4-7
 // store dV, 8-11 dK.
 // TMEM columns: dV [0,d) dK [d,2d) R1 [2d,2d+128) R2 [2d+128,2d+256); at d = 64
-// the untransposed dQ tile has its own columns [384, 448).
+// the untransposed dQ tile has its own columns [384, 448), and copies of K_j
+// and V_j (the A operands of S^T and dP^T) sit in [448, 480) and [480, 512).
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -141,6 +142,12 @@ struct BwdShape {
   // so the next dP^T does not wait for the dQ warpgroup to read dQ out.
   static constexpr uint32_t kColDQ = kTmaDQ ? 384u : uint32_t(2 * D + 128);
   static constexpr uint32_t kColDV = 0, kColDK = D, kColR1 = 2 * D, kColR2 = 2 * D + 128;
+  // d = 64 also leaves [448, 512) free: K_j and V_j are copied there once, as
+  // bf16 pairs (lane = key row), and S^T = K Q^T, dP^T = V dO^T take them as
+  // the TMEM A operand, so these two products read only Q / dO from shared
+  // memory (the shared-memory data path is the busiest unit of this kernel).
+  static constexpr bool kTmemKV = (D == 64);
+  static constexpr uint32_t kColKt = 448, kColVt = 480;
   // Exponentials per 8 pairs computed on the FMA pipe on fully unmasked tiles.
   // None: measured on B200, moving 2/8 or 3/8 of them off MUFU made this
   // kernel slower (12-20 % at d = 64), the extra FMA-pipe instructions cost
@@ -154,6 +161,7 @@ struct BwdBarriers {
   uint64_t qdo_full[NST];
   uint64_t qdo_empty[NST];
   uint64_t s_ready, dp_ready, p_ready, ds_ready, ds_free, dq_ready, dq_free, final_;
+  uint64_t kv_tmem;                          // d = 64: K_j, V_j copied into TMEM (8 warps)
   uint64_t dq_staged[2], dq_stage_free[2];   // TMA-reduced dQ (d = 64)
   uint32_t tmem_base;
   uint32_t abort;
@@ -230,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->p_ready, 8);
     mbar_init(&bars->ds_ready, 8);
     mbar_init(&bars->ds_free, 1);
+    mbar_init(&bars->kv_tmem, 8);
     mbar_init(&bars->dq_ready, 1);
     mbar_init(&bars->dq_free, 4);
     mbar_init(&bars->final_, 1);
@@ -301,18 +310,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t ddS_mn = sdesc_sw128(smem_u32(sdS), 16384, 1024);// dS^T, MN-major (B of dQ^T)
     constexpr uint64_t kTileD = uint64_t(S::kTileBytes >> 4);
     // X^T tile = A_tile B_tile^T over d, both K-major (S^T = K Q^T, dP^T = V dO^T).
-    auto issue_xt = [&](uint32_t d_tmem, uint64_t a, uint64_t b) {
+    // d = 64: A (K or V) from its TMEM copy instead of shared memory.
+    auto issue_xt = [&](uint32_t d_tmem, uint64_t a, uint32_t a_tmem, uint64_t b) {
 #pragma unroll
       for (int ks = 0; ks < S::kKSteps; ++ks) {
         const uint64_t off = uint64_t(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
-        mma_f16_ss_e(d_tmem, a + off, b + off, S::kIdSS, ks > 0 ? 1u : 0u);
+        if constexpr (S::kTmemKV)
+          mma_f16_ts_e(d_tmem, a_tmem + uint32_t(ks * 8), b + off, S::kIdSS, ks > 0 ? 1u : 0u);
+        else
+          mma_f16_ss_e(d_tmem, a + off, b + off, S::kIdSS, ks > 0 ? 1u : 0u);
       }
     };
     bool ok = mbar_wait_warp(&bars->kv_full, 0, wc, WAIT_BWD_KV) &&
-              mbar_wait_warp(&bars->qdo_full[0], 0, wc, WAIT_BWD_QDO);
+              mbar_wait_warp(&bars->qdo_full[0], 0, wc, WAIT_BWD_QDO) &&
+              (!S::kTmemKV || mbar_wait_warp(&bars->kv_tmem, 0, wc, WAIT_BWD_KV));
     if (ok) {
       tc_fence_after();
-      issue_xt(tR1, dK_k, dQ_k);                       // S^T_0
+      issue_xt(tR1, dK_k, tmem + S::kColKt, dQ_k);     // S^T_0
       tc_commit_e(&bars->s_ready);
       for (int it = 0; it < n_iter; ++it) {
         const int s = it % NST;
@@ -321,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait_warp(&bars->dq_free, (it - 1) & 1, wc, WAIT_BWD_DQ_FREE)) { ok = false; break; }
           tc_fence_after();
         }
-        issue_xt(tR2, dV_k, ddO_k + st);               // dP^T_it
+        issue_xt(tR2, dV_k, tmem + S::kColVt, ddO_k + st);   // dP^T_it
         tc_commit_e(&bars->dp_ready);
         if (!mbar_wait_warp(&bars->p_ready, it & 1, wc, WAIT_BWD_P)) { ok = false; break; }
         tc_fence_after();
@@ -335,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int sn = (it + 1) % NST;
           if (!mbar_wait_warp(&bars->qdo_full[sn], ((it + 1) / NST) & 1, wc, WAIT_BWD_QDO)) { ok = false; break; }
           tc_fence_after();
-          issue_xt(tR1, dK_k, dQ_k + uint64_t(sn) * kTileD);
+          issue_xt(tR1, dK_k, tmem + S::kColKt, dQ_k + uint64_t(sn) * kTileD);
           tc_commit_e(&bars->s_ready);
         }
         if (!mbar_wait_warp(&bars->ds_ready, it & 1, wc, WAIT_BWD_DS)) { ok = false; break; }
@@ -392,6 +406,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool kv_tile_full = (j + 1) * kTile <= N;
     uint8_t* ds_row = sdS + h * 16384 + (c >> 3) * 1024 + (c & 7) * 128;
     bool ok = true;
+    if constexpr (S::kTmemKV) {
+      // Group 0 copies row c of K_j, group 1 row c of V_j, into TMEM: the
+      // 128-byte swizzled row holds d = 8u .. 8u+7 in 16-byte unit u ^ (c % 8).
+      ok = mbar_wait_warp(&bars->kv_full, 0, wc, WAIT_BWD_KV);
+      if (ok) {
+        const uint8_t* row = (h == 0 ? sK : sV) + (c >> 3) * 1024 + (c & 7) * 128;
+        uint32_t r[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 x = *reinterpret_cast<const uint4*>(row + ((u ^ (c & 7)) << 4));
+          r[4 * u] = x.x;
+          r[4 * u + 1] = x.y;
+          r[4 * u + 2] = x.z;
+          r[4 * u + 3] = x.w;
+        }
+        tmem_st_x32(lane_base + (h == 0 ? S::kColKt : S::kColVt), r);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->kv_tmem);
+      }
+    }
     for (int it = 0; it < n_iter && ok; ++it) {
       const int s = it % NST;
       const int i = i_begin + it;
