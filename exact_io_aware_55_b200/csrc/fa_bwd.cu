@@ -16,12 +16,13 @@
 //   bwd_kernel   one CTA per (key tile j, batch-head); K_j, V_j stay in shared
 //                memory, dK_j and dV_j accumulate in TMEM, and the CTA walks the
 //                query tiles i (from the diagonal when causal):
-//                  S^T = K_j Q_i^T      -> TMEM R1       (tcgen05, smem x smem)
-//                  dP^T = V_j dO_i^T    -> TMEM R2
+//                  S^T = K_j Q_i^T      -> TMEM R1       (tcgen05; K from TMEM at
+//                  dP^T = V_j dO_i^T    -> TMEM R2        d = 64, else smem)
 //                  P^T = exp2(S^T c - LSE2_i)  written back over R1 as bf16
 //                  dV_j += P^T dO_i     (A = P^T from TMEM)
-//                  dS^T = scale P^T o (dP^T - D_i) -> shared memory (bf16, swizzled)
-//                  dK_j += dS^T Q_i     (A = dS^T, K-major)
+//                  dS^T = P^T o (dP^T - D_i) -> shared memory (bf16, swizzled)
+//                                       and over the dP^T columns of R2
+//                  dK_j += dS^T Q_i     (A = dS^T from TMEM)
 //                  d = 128: dQ_i^T = K_j^T dS^T -> TMEM R2 (both operands read
 //                           MN-major from the K tile and the dS^T bytes), then
 //                           fp32 red.add into the workspace accumulator, one
@@ -306,7 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), 16384, 1024);  // Q stages, MN-major (B of dK)
     const uint64_t ddO_mn = sdesc_sw128(smem_u32(sdO), 16384, 1024);// dO stages, MN-major (B of dV)
     const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), 16384, 1024);  // K tile, MN-major (A of dQ^T)
-    const uint64_t ddS_k = sdesc_sw128(smem_u32(sdS), 16, 1024);    // dS^T, K-major (A of dK)
     const uint64_t ddS_mn = sdesc_sw128(smem_u32(sdS), 16384, 1024);// dS^T, MN-major (B of dQ^T)
     constexpr uint64_t kTileD = uint64_t(S::kTileBytes >> 4);
     // X^T tile = A_tile B_tile^T over d, both K-major (S^T = K Q^T, dP^T = V dO^T).
@@ -354,13 +354,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!mbar_wait_warp(&bars->ds_ready, it & 1, wc, WAIT_BWD_DS)) { ok = false; break; }
         tc_fence_after();
-        // dK += dS^T Q: A = dS^T K-major (rows = keys, 128 queries), B = Q MN-major.
+        // dK += dS^T Q: A = dS^T from TMEM R2 (bf16; queries 0-63 in columns
+        // [0,32), 64-127 in [64,96)), B = Q MN-major; 16 queries per step.
 #pragma unroll
-        for (int kt = 0; kt < 8; ++kt) {
-          const uint64_t off = uint64_t(((kt >> 2) * 16384 + (kt & 3) * 32) >> 4);
-          mma_f16_ss_e(tmem + S::kColDK, ddS_k + off, dQ_mn + st + uint64_t(kt * 128), S::kIdKmaj,
-                       (it > 0 || kt > 0) ? 1u : 0u);
-        }
+        for (int kt = 0; kt < 8; ++kt)
+          mma_f16_ts_e(tmem + S::kColDK, tR2 + uint32_t(kt * 8 + (kt >= 4 ? 32 : 0)), dQ_mn + st + uint64_t(kt * 128),
+                       S::kIdKmaj, (it > 0 || kt > 0) ? 1u : 0u);
         // dQ^T = K^T dS^T: A = K read MN-major (M = d), B = the dS^T bytes read
         // MN-major (N = queries); 16 keys per step.  The transposed product puts
         // d on the TMEM lanes, so each dQ row update is one coalesced line.
@@ -498,8 +497,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = 0; u < 4; ++u)
           *reinterpret_cast<uint4*>(ds_row + (((4 * q + u) ^ (c & 7)) << 4)) =
               make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        // The same bf16 pairs into R2 over dP^T columns already read: the A
+        // operand of dK, so dK reads only Q from shared memory.
+        tmem_st_x16(tdP + 16 * q, w);
       }
       fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
