@@ -69,6 +69,18 @@ def test_fwd_config_b4_h16_n2048_d64_full():
     gu.assert_o_lse(o, lse, o_ref, lse_ref)
 
 
+def test_fwd_d64_persistent_items_ragged_b2_h40_n1000():
+    """d = 64, non-causal: 80 heads x 4 Q-tile pairs = 320 pairs on 148 SMs.
+    The last 24 pairs are split into 48 single-tile items (344 items), so each
+    persistent CTA takes two or three items, single tiles among them.  Every
+    head's last Q tile and last K/V tile are ragged (104 of 128 rows), and the
+    output buffers are guarded against writes outside them."""
+    inp = synth.attention_inputs(2, 40, 1000, 64, seed=1241, with_grad=False)
+    o, lse, scale = _run_fwd(inp, False, guarded=True)
+    o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], scale, False)
+    gu.assert_o_lse(o, lse, o_ref, lse_ref)
+
+
 def _sampled_check(B, H, N, d, causal, seed, q_mult=1.0, n_heads=3, n_rows=24):
     inp = synth.attention_inputs(B, H, N, d, seed=seed, q_mult=q_mult, with_grad=False, want_f64=False)
     o, lse, scale = _run_fwd(inp, causal)
