@@ -3,8 +3,9 @@
 // Method (explainers.rudrite.com "flash-attention-anatomy", Q&A "What is
 // online softmax and how does tiling keep it exact?"): the same tiled online
 // softmax as the d = 128 kernel in fa_fwd.cu (lazy rescaling included), with
-// the same warp roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer,
-// warps 4-11 two softmax warpgroups, one per 128-row Q tile.
+// similar warp roles: warp 0 TMA producer, warps 1 and 2 the MMA issuers of Q
+// tile 0 and Q tile 1 (warp 1 also owns TMEM), warps 4-11 two softmax
+// warpgroups, one per 128-row Q tile.
 //
 // At d = 64 the two MMAs of a tile take about half as long as its softmax, so
 // the kernel is bound by how busy the softmax warps are kept.
@@ -114,12 +115,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->q_full[b], 1);
-      mbar_init(&bars->q_empty[b], 1);
+      mbar_init(&bars->q_empty[b], kNQT);
     }
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->kv_empty[s], kNQT);
     }
     for (int g = 0; g < kNQT; ++g) {
       mbar_init(&bars->s_full[g], 1);
@@ -176,101 +177,105 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d_hint_e(sV + s * kD64Tile, &tmV, &bars->v_full[s], 0, j * kBN, bh, pol_kv);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
     // ----------------------------------------------------------------- MMA
-    // Per K/V tile j of an item: S_g(j+1) for each slot once the softmax
-    // holds S_g(j), then O_g += P_g(j) V_j as each P_g(j) is ready.
+    // One warp per slot: warp 1 issues every MMA of Q tile 0, warp 2 of Q
+    // tile 1, so neither softmax warpgroup waits on the other (at an item
+    // boundary, or when one runs a tile ahead).  Per K/V tile j of an item:
+    // S_g(j+1) once the softmax holds S_g(j), then O_g += P_g(j) V_j.  Both
+    // warps release every K/V stage and Q buffer (kv_empty and q_empty count
+    // two arrivals).  A warp whose slot has no work on a tile or an item still
+    // waits for that tile's (item's) load before releasing it, so its release
+    // can never count towards the previous use of the stage (buffer).
+    const int g = warp - 1;
     const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);       // K-major
     const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);       // K-major
     const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16384, 1024);    // MN-major
     constexpr uint64_t kTileD = uint64_t(kD64Tile >> 4);
     constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
     constexpr uint32_t kIdPV = idesc_bf16(128, 64, false, true);
-    auto issue_s = [&](int g, int qb, int s) {
+    auto issue_s = [&](int qb, int s) {
       const uint64_t a = dQ0 + uint64_t(qb * kNQT + g) * kTileD, b = dK0 + uint64_t(s) * kTileD;
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)   // 16 of the 64 head dims per step
         mma_f16_ss_e(tmem + uint32_t(g * 128), a + uint64_t(ks * 2), b + uint64_t(ks * 2), kIdS, ks > 0 ? 1u : 0u);
     };
-    auto issue_pv = [&](int g, int s, bool acc) {
+    auto issue_pv = [&](int s, bool acc) {
       const uint64_t b = dV0 + uint64_t(s) * kTileD;
 #pragma unroll
       for (int kt = 0; kt < 8; ++kt)   // 16 keys per step
         mma_f16_ts_e(tmem + kD64ColO + uint32_t(g * 64), tmem + kD64ColP + uint32_t(g * 64 + kt * 8),
                      b + uint64_t(kt * 128), kIdPV, (acc || kt > 0) ? 1u : 0u);
     };
-    int kv_c = 0;                    // K/V tiles consumed so far
-    int n_s[kNQT] = {0, 0};          // S tiles issued per slot
-    int n_p[kNQT] = {0, 0};          // P tiles consumed per slot
+    int kv_c = 0;                    // K/V tiles walked so far (ring position)
+    int n_s = 0;                     // S tiles issued for this slot
+    int n_p = 0;                     // P tiles consumed for this slot
     int n = 0;                       // items taken
     bool ok = true;
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++n) {
       int bh, pair, only, q0[kNQT], T[kNQT];
       fwd_item<CAUSAL>(w, args, n_pairs, bh, pair, only);
 #pragma unroll
-      for (int g = 0; g < kNQT; ++g) fwd_slot<CAUSAL>(pair, only, g, N, n_kv, q0[g], T[g]);
+      for (int gg = 0; gg < kNQT; ++gg) fwd_slot<CAUSAL>(pair, only, gg, N, n_kv, q0[gg], T[gg]);
       const int Tmax = max(T[0], T[1]);
+      const int Tg = (g == 0) ? T[0] : T[1];
       const int qb = n & 1;
-      if (!mbar_wait_warp(&bars->q_full[qb], (n >> 1) & 1, wc, WAIT_FWD_Q) ||
-          !mbar_wait_warp(&bars->k_full[kv_c % NST], (kv_c / NST) & 1, wc, WAIT_FWD_K)) {
+      if (!mbar_wait_warp(&bars->q_full[qb], (n >> 1) & 1, wc, WAIT_FWD_Q)) {
         ok = false;
         break;
       }
-#pragma unroll
-      for (int g = 0; g < kNQT; ++g) {
-        if (T[g] == 0 || !ok) continue;
-        if (n_s[g] > 0 && !mbar_wait_warp(&bars->s_free[g], (n_s[g] - 1) & 1, wc, WAIT_FWD_S_FREE)) {
-          ok = false;
-          continue;
-        }
-        tc_fence_after();
-        issue_s(g, qb, kv_c % NST);
-        tc_commit_e(&bars->s_full[g]);
-        ++n_s[g];
-      }
-      for (int j = 0; j < Tmax && ok; ++j, ++kv_c) {
-        const int s = kv_c % NST;
-        bool k_next_ready = false;
-#pragma unroll
-        for (int g = 0; g < kNQT; ++g) {
-          if (j + 1 >= T[g] || !ok) continue;
-          if (!mbar_wait_warp(&bars->s_free[g], (n_s[g] - 1) & 1, wc, WAIT_FWD_S_FREE)) {
-            ok = false;
-            continue;
-          }
-          if (!k_next_ready) {
-            const int c1 = kv_c + 1;
-            if (!mbar_wait_warp(&bars->k_full[c1 % NST], (c1 / NST) & 1, wc, WAIT_FWD_K)) {
-              ok = false;
-              continue;
-            }
-            k_next_ready = true;
-          }
-          tc_fence_after();
-          issue_s(g, qb, (kv_c + 1) % NST);
-          tc_commit_e(&bars->s_full[g]);
-          ++n_s[g];
-        }
-        if (!ok || !mbar_wait_warp(&bars->v_full[s], (kv_c / NST) & 1, wc, WAIT_FWD_V)) {
+      if (Tg > 0) {
+        if (!mbar_wait_warp(&bars->k_full[kv_c % NST], (kv_c / NST) & 1, wc, WAIT_FWD_K) ||
+            (n_s > 0 && !mbar_wait_warp(&bars->s_free[g], (n_s - 1) & 1, wc, WAIT_FWD_S_FREE))) {
           ok = false;
           break;
         }
-#pragma unroll
-        for (int g = 0; g < kNQT; ++g) {
-          if (j >= T[g] || !ok) continue;
-          if (!mbar_wait_warp(&bars->p_full[g], n_p[g] & 1, wc, WAIT_FWD_P)) {
+        tc_fence_after();
+        issue_s(qb, kv_c % NST);
+        tc_commit_e(&bars->s_full[g]);
+        ++n_s;
+      }
+      for (int j = 0; j < Tmax; ++j, ++kv_c) {
+        const int s = kv_c % NST;
+        if (j < Tg) {
+          if (j + 1 < Tg) {
+            const int c1 = kv_c + 1;
+            if (!mbar_wait_warp(&bars->s_free[g], (n_s - 1) & 1, wc, WAIT_FWD_S_FREE) ||
+                !mbar_wait_warp(&bars->k_full[c1 % NST], (c1 / NST) & 1, wc, WAIT_FWD_K)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(qb, c1 % NST);
+            tc_commit_e(&bars->s_full[g]);
+            ++n_s;
+          }
+          if (!mbar_wait_warp(&bars->v_full[s], (kv_c / NST) & 1, wc, WAIT_FWD_V) ||
+              !mbar_wait_warp(&bars->p_full[g], n_p & 1, wc, WAIT_FWD_P)) {
             ok = false;
-            continue;
+            break;
           }
           tc_fence_after();
-          issue_pv(g, s, j > 0);
+          issue_pv(s, j > 0);
           tc_commit_e(&bars->pv_done[g]);
-          ++n_p[g];
-          if (j + 1 == T[g]) tc_commit_e(&bars->o_final[g]);
+          ++n_p;
+          if (j + 1 == Tg) tc_commit_e(&bars->o_final[g]);
+          tc_commit_e(&bars->kv_empty[s]);
+        } else {
+          // This slot has no work on tile j: release the stage once it is filled.
+          if (!mbar_wait_warp(&bars->v_full[s], (kv_c / NST) & 1, wc, WAIT_FWD_V)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive(&bars->kv_empty[s]);
         }
-        tc_commit_e(&bars->kv_empty[s]);
       }
-      if (ok) tc_commit_e(&bars->q_empty[qb]);
+      if (!ok) break;
+      if (Tg > 0) {
+        tc_commit_e(&bars->q_empty[qb]);
+      } else if (lane == 0) {
+        mbar_arrive(&bars->q_empty[qb]);
+      }
     }
     // Let the last commits land before the CTA can exit.
     if (ok && n > 0)
