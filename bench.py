@@ -19,6 +19,7 @@ bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import importlib.util
 import json
 import math
 import os
@@ -378,18 +379,34 @@ def run_case(args):
     print(json.dumps(line), flush=True)
 
 
+def kernel_source_digest(files) -> str:
+    """sha256 over the named library sources (paths relative to the package's
+    csrc/ directory) and the build flags: the sources a kernel is built from."""
+    import hashlib
+    spec = importlib.util.spec_from_file_location("_fa_build", os.path.join(ROOT, "exact_io_aware_55_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    h = hashlib.sha256()
+    for name in files:
+        h.update(name.encode())
+        h.update(open(os.path.normpath(os.path.join(build.CSRC, name)), "rb").read())
+    h.update(" ".join(build.ARCH + build.FLAGS).encode())
+    return h.hexdigest()
+
+
 def committed_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the library build that is loaded now (same source digest); else None."""
+    the sources the kernel is built from now (same digest over the files the
+    entry lists, and the same build flags); else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    digest_path = os.path.join(ROOT, "exact_io_aware_55_b200", "libfa.so.sha256")
-    if not (os.path.exists(path) and os.path.exists(digest_path)):
+    if not os.path.exists(path):
         return None
     try:
-        data = json.load(open(path))
-        digest = open(digest_path).read().strip()
-        ent = data.get(kernel, {})
-        if ent.get("source_digest") == digest and ent.get("workload") == workload:
+        ent = json.load(open(path)).get(kernel, {})
+        files = ent.get("source_files")
+        if not files or ent.get("workload") != workload:
+            return None
+        if ent.get("source_digest") == kernel_source_digest(files):
             return ent.get("dram_bytes_per_launch")
     except (OSError, ValueError):
         return None
