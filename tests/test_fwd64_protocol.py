@@ -4,9 +4,10 @@ The model runs the roles of ``fwd64_kernel`` (csrc/fa_fwd64.cu) as coroutines:
 the TMA producer, one MMA-issuing warp per Q-tile slot, the two softmax
 warpgroups, the TMA engine (loads complete asynchronously) and the in-order
 tensor pipe (MMAs and ``tcgen05.commit`` arrivals execute in issue order).
-A random scheduler interleaves them.  Each mbarrier wait names the completion
-it intends (the kernel's parity expression); the model applies the hardware
-rule (a parity wait passes once the barrier's phase parity differs) and checks:
+A random scheduler with per-run random speeds interleaves them.  Each mbarrier
+wait names the completion it intends (the kernel's parity expression); the
+model applies the hardware rule (a parity wait passes once the barrier's phase
+parity differs) and checks:
 
 * no deadlock;
 * every wait that passes sees exactly its intended completion (no parity
@@ -64,6 +65,7 @@ class Model:
         self.p_full = [B("p_full0", 1), B("p_full1", 1)]
         self.pv_done = [B("pv_done0", 1), B("pv_done1", 1)]
         self.o_final = [B("o_final0", 1), B("o_final1", 1)]
+        self.speeds = {}
         self.pipe = []          # in-order tensor pipe: ("mma", info) | ("commit", bar)
         self.tma = []           # outstanding loads: bars to arrive on
         # buffer bookkeeping
@@ -75,6 +77,13 @@ class Model:
     # ------------------------------------------------------------------ roles
     def wait(self, bar, k):
         return ("wait", bar, k)
+
+    def speed(self, actor):
+        """Per-run random speed of each role and engine (log-uniform over three
+        decades), so that some runs starve one of them for long stretches."""
+        if actor not in self.speeds:
+            self.speeds[actor] = 10.0 ** self.rng.uniform(-3.0, 0.0)
+        return self.speeds[actor]
 
     def producer(self):
         kv_c = 0
@@ -197,7 +206,7 @@ class Model:
                     return
                 waits = {nm: (pending[nm][1].name, pending[nm][2]) for nm in roles}
                 raise Violation(f"deadlock: {waits}")
-            c = self.rng.choice(choices)
+            c = self.rng.choices(choices, weights=[self.speed(x) for x in choices])[0]
             if c == "tma":
                 self.tma.pop(self.rng.randrange(len(self.tma))).arrive()
             elif c == "pipe":
