@@ -1,9 +1,10 @@
-"""CPU model of the synchronisation protocol of the d = 64 backward main kernel.
+"""CPU model of the synchronisation protocol of the backward main kernel.
 
-The model runs the roles of ``bwd_kernel<64, CAUSAL, dQ>`` (csrc/fa_bwd.cu,
-the path with the fp32 dQ accumulator) as coroutines: the TMA producer, the
-MMA warp, the two P/dS warpgroups, the dQ warpgroup with its TMA bulk
-reductions, the TMA engine (loads and reduction reads complete
+The model runs the roles of ``bwd_kernel<D, CAUSAL, dQ>`` (csrc/fa_bwd.cu,
+the path with the fp32 dQ accumulator), for d = 64 and d = 128, as
+coroutines: the TMA producer, the MMA warp, the two P/dS warpgroups, the dQ
+warpgroup (d = 64: TMA bulk reductions through two staging tiles; d = 128:
+dQ^T read from R2 and added with red.global.add), the TMA engine (loads and reduction reads complete
 asynchronously, reductions in issue order) and the in-order tensor pipe (MMAs
 and ``tcgen05.commit`` arrivals execute in issue order).  A random scheduler
 with per-run random speeds interleaves them.  Each mbarrier wait names the
@@ -12,7 +13,9 @@ completion it intends (the kernel's parity expression), and the model checks:
 * no deadlock, and every wait that passes sees exactly its intended completion;
 * no TMEM region, shared-memory buffer or ring stage is rewritten while a read
   of its previous contents is pending, and no product reads a region before
-  its contents are written: K and V copied into TMEM before the first S^T;
+  its contents are written: K and V copied into TMEM before the first S^T
+  (d = 64); at d = 128, dQ^T_i over dS^T_i in R2 only after dK_i used it, and
+  dP^T_(i+1) over dQ^T_i only after the dQ group read it;
   S^T_(i+1) over P^T_i only after dV used it; dP^T_(i+1) over dS^T_i only
   after dK used it; P^T_i and dS^T_i written only after their TMEM columns
   were read; dS^T_i in shared memory only after dQ_(i-1) read it; dQ_i into
@@ -48,8 +51,8 @@ class Violation(Exception):
 
 
 class Model:
-    def __init__(self, n_iter, rng, plant=None):
-        self.n, self.rng, self.plant = n_iter, rng, plant
+    def __init__(self, n_iter, rng, plant=None, d=64):
+        self.n, self.rng, self.plant, self.d = n_iter, rng, plant, d
         B = Bar
         self.kv_full = B("kv_full", 1)
         self.kv_tmem = B("kv_tmem", 2)
@@ -95,11 +98,14 @@ class Model:
     def mma(self):
         yield self.wait(self.kv_full, 0)
         yield self.wait(self.qdo_full[0], 0)
-        yield self.wait(self.kv_tmem, 0)
+        if self.d == 64:
+            yield self.wait(self.kv_tmem, 0)
         self.pipe.append(("S", 0))
         self.pipe.append(("commit", self.s_ready))
         for it in range(self.n):
             s = it % NST
+            if self.d == 128 and it > 0 and self.plant != "no_dq_free":
+                yield self.wait(self.dq_free, it - 1)     # dP^T reuses R2, where dQ^T was
             self.pipe.append(("dP", it))
             self.pipe.append(("commit", self.dp_ready))
             yield self.wait(self.p_ready, it)
@@ -110,7 +116,7 @@ class Model:
                 self.pipe.append(("commit", self.s_ready))
             yield self.wait(self.ds_ready, it)
             self.pipe.append(("dK", it))
-            if it > 0 and self.plant != "no_dq_free":
+            if self.d == 64 and it > 0 and self.plant != "no_dq_free":
                 yield self.wait(self.dq_free, it - 1)
             self.pipe.append(("dQ", it))
             self.pipe.append(("commit", self.dq_ready))
@@ -120,9 +126,10 @@ class Model:
         yield self.wait(self.final_, 0)
 
     def pds(self, h):
-        yield self.wait(self.kv_full, 0)
-        self.kv_copied += 1
-        self.kv_tmem.arrive()
+        if self.d == 64:
+            yield self.wait(self.kv_full, 0)
+            self.kv_copied += 1
+            self.kv_tmem.arrive()
         for it in range(self.n):
             s = it % NST
             yield self.wait(self.qdo_full[s], it // NST)
@@ -147,6 +154,12 @@ class Model:
             raise Violation("epilogue before every product executed")
 
     def dq_group(self):
+        if self.d == 128:                                # dQ^T from R2, then red.global.add
+            for it in range(self.n):
+                yield self.wait(self.dq_ready, it)
+                self.dq_read += 1
+                self.dq_free.arrive()
+            return
         for it in range(self.n):
             b = it & 1
             yield self.wait(self.dq_ready, it)
@@ -176,13 +189,15 @@ class Model:
         it = x
         s = it % NST
         if op == "S":
-            if self.kv_copied < 2:
+            if self.d == 64 and self.kv_copied < 2:
                 raise Violation("S^T issued before K and V were copied into TMEM")
             if it > 0 and (self.exec["dV"] < it or min(self.p_done) < it):
                 raise Violation(f"S^T_{it} overwrote P^T_{it - 1} before it was used")
         elif op == "dP":
             if it > 0 and (self.exec["dK"] < it or min(self.ds_done) < it):
                 raise Violation(f"dP^T_{it} overwrote dS^T_{it - 1} before it was used")
+            if self.d == 128 and self.dq_read < it:
+                raise Violation(f"dP^T_{it} overwrote dQ^T_{it - 1} before the dQ group read it")
         elif op == "dV":
             if min(self.p_done) < it + 1:
                 raise Violation(f"dV_{it} read P^T before it was written")
@@ -191,6 +206,8 @@ class Model:
                 raise Violation(f"{op}_{it} read dS^T before it was written")
             if op == "dQ" and self.dq_read < it:
                 raise Violation(f"dQ_{it} overwrote dQ_{it - 1} before the dQ group read it")
+            if op == "dQ" and self.d == 128 and self.exec["dK"] < it + 1:
+                raise Violation(f"dQ^T_{it} overwrote dS^T_{it} in R2 before dK_{it} read it")
         self.exec[op] += 1
         if op in ("S", "dP", "dV", "dK"):
             self.stage_reads[(s, it)] = self.stage_reads.get((s, it), 0) + 1
@@ -236,19 +253,21 @@ class Model:
         raise Violation("step limit")
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("n_iter", [1, 2, 3, 5, 16])
-def test_protocol_holds_under_random_interleavings(n_iter):
+def test_protocol_holds_under_random_interleavings(n_iter, d):
     for seed in range(80):
-        Model(n_iter, random.Random(seed)).run()
+        Model(n_iter, random.Random(seed), d=d).run()
 
 
-def test_protocol_model_catches_a_planted_missing_wait():
+@pytest.mark.parametrize("d", [64, 128])
+def test_protocol_model_catches_a_planted_missing_wait(d):
     # Without its dq_free wait the MMA warp may overwrite dQ_(i-1) in TMEM
-    # before the dQ group has read it out.
+    # (d = 64) or dQ^T_(i-1) in R2 (d = 128) before the dQ group has read it.
     caught = 0
     for seed in range(200):
         try:
-            Model(4, random.Random(seed), plant="no_dq_free").run()
+            Model(4, random.Random(seed), plant="no_dq_free", d=d).run()
         except Violation:
             caught += 1
     assert caught > 0
