@@ -16,7 +16,7 @@ from ._lib import FA_OK, FAError, LIB_PATH, STATUS_CODES, STATUS_NAMES, check, l
 
 __all__ = [
     "FAError", "LIB_PATH", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size",
-    "fa_device_status", "fa_fwd_decode", "fa_fwd_decode_workspace_size", "attention_decode",
+    "fa_bwd_events", "fa_fwd_plan", "fa_get_device_status", "fa_device_status", "fa_fwd_decode", "fa_fwd_decode_workspace_size", "attention_decode",
     "fa_fwd_standard", "fa_fwd_standard_workspace_size", "attention_forward_standard",
     "fa_watchdog_selftest", "attention_forward", "attention_backward", "attention_forward_fp8", "lib",
     "STATUS_NAMES", "STATUS_CODES", "strerror",
@@ -85,6 +85,29 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, workspac
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                      B, H, N, d, float(scale), int(bool(causal)), _ptr(workspace), wbytes, _stream_ptr(stream)))
+
+
+def fa_bwd_events(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, workspace, events,
+                  stream=None) -> None:
+    """fa_bwd that also records four torch.cuda.Event objects on the stream:
+    before the preprocess, before and after the main kernel, after the last launch."""
+    B, H, N, d = _shape(q)
+    _check_tensors((B, H, N, d), torch.bfloat16, q, k, v, o, do, dq, dk, dv)
+    _check_tensors((B, H, N), torch.float32, lse)
+    if len(events) != 4:
+        raise ValueError("fa_bwd_events takes four events")
+    arr = (ctypes.c_void_p * 4)(*(int(e.cuda_event) for e in events))
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.fa_bwd_events(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                            B, H, N, d, float(scale), int(bool(causal)), _ptr(workspace), wbytes, arr,
+                            _stream_ptr(stream)))
+
+
+def fa_fwd_plan(B: int, H: int, N: int, d: int, causal: bool):
+    """(ctas, items, pair_items) of the forward's launch for this shape."""
+    c, it, pi = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    check(lib.fa_fwd_plan(B, H, N, d, int(bool(causal)), ctypes.byref(c), ctypes.byref(it), ctypes.byref(pi)))
+    return c.value, it.value, pi.value
 
 
 def fa_bwd_deterministic(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, workspace,

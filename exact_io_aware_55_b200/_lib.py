@@ -58,6 +58,13 @@ def _load() -> ctypes.CDLL:
     lib.fa_fwd_standard.restype = i
     lib.fa_fwd_standard_workspace_size.argtypes = [i, i, i, i]
     lib.fa_fwd_standard_workspace_size.restype = sz
+    lib.fa_bwd_events.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz,
+                                  ctypes.POINTER(vp), vp]
+    lib.fa_bwd_events.restype = i
+    lib.fa_fwd_plan.argtypes = [i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i), ctypes.POINTER(i)]
+    lib.fa_fwd_plan.restype = i
+    lib.fa_get_device_status.argtypes = [vp]
+    lib.fa_get_device_status.restype = i
     lib.fa_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_bwd_deterministic.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]

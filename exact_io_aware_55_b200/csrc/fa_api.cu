@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -134,7 +135,7 @@ bool make_map_p(CUtensorMap* map, const void* base, int Np, int N, int BH) {
 fa_status check_shape(int B, int H, int N, int d, float scale, int causal, bool* empty) {
   if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
-  if (!(std::isfinite(scale) && scale > 0.0f)) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale >= 0.0f)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(B) * H;
   if (BH > 65535) return FA_ERR_UNSUPPORTED;  // grid.y limit of the launch shapes
@@ -247,7 +248,7 @@ int sm_count() {
 fa_status check_decode(int B, int H, int Nq, int Nk, int d, float scale, int causal, bool* empty) {
   if (B < 0 || H < 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
-  if (!(std::isfinite(scale) && scale > 0.0f)) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale >= 0.0f)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (Nq > kDecodeMaxNq) return FA_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(B) * H;
@@ -303,6 +304,26 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   return fwd_common(q, k, v, o, lse, B, H, N, d, scale, causal, stream, false, 1.f, 1.f, 1.f);
 }
 
+fa_status fa_fwd_plan(int B, int H, int N, int d, int causal, int* ctas, int* items, int* pair_items) {
+  bool empty = false;
+  fa_status st = check_shape(B, H, N, d, 1.0f, causal, &empty);
+  if (st != FA_OK) return st;
+  if (!ctas || !items || !pair_items) return FA_ERR_INVALID_ARG;
+  *ctas = *items = *pair_items = 0;
+  if (empty) return FA_OK;
+  const long long BH = static_cast<long long>(B) * H;
+  if (!grid_fits(BH, N)) return FA_ERR_UNSUPPORTED;
+  const long long pairs = BH * ((static_cast<long long>(N) + 2 * 128 - 1) / (2 * 128));
+  const long long pair_blocks = causal ? pairs : fwd_pair_blocks(BH, N);
+  const long long n_items = pair_blocks + 2 * (pairs - pair_blocks);
+  // d = 64 non-causal runs persistent CTAs (at most one per SM) over the items
+  const long long n_ctas = (d == 64 && !causal) ? std::min<long long>(n_items, sm_count()) : n_items;
+  *ctas = static_cast<int>(n_ctas);
+  *items = static_cast<int>(n_items);
+  *pair_items = static_cast<int>(pair_blocks);
+  return FA_OK;
+}
+
 fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_descale, float k_descale,
                      float v_descale, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
                      void* stream) {
@@ -319,21 +340,30 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
 namespace {
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                      void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
-                     void* workspace, size_t workspace_bytes, void* stream, bool deterministic);
+                     void* workspace, size_t workspace_bytes, void* stream, bool deterministic,
+                     void* const* events);
 }  // namespace
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                  void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_common(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes, stream,
-                    false);
+                    false, nullptr);
+}
+
+fa_status fa_bwd_events(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                        void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                        void* workspace, size_t workspace_bytes, void* const* events, void* stream) {
+  if (!events || !events[0] || !events[1] || !events[2] || !events[3]) return FA_ERR_INVALID_ARG;
+  return bwd_common(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes, stream,
+                    false, events);
 }
 
 fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,
                                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                                float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_common(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes, stream,
-                    true);
+                    true, nullptr);
 }
 
 }  // extern "C"
@@ -341,7 +371,8 @@ fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, cons
 namespace {
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                      void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
-                     void* workspace, size_t workspace_bytes, void* stream, bool deterministic) {
+                     void* workspace, size_t workspace_bytes, void* stream, bool deterministic,
+                     void* const* events) {
   bool empty = false;
   fa_status st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK) return st;
@@ -381,7 +412,8 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   CUtensorMap tdq;
   if (!make_map_dq(&tdq, a.dq_acc, d, N, BH)) return FA_ERR_LAUNCH;
   return launch_status(
-      fa::launch_bwd(tq, tk, tv, tdo, tdq, a, d, causal != 0, deterministic, static_cast<cudaStream_t>(stream)));
+      fa::launch_bwd(tq, tk, tv, tdo, tdq, a, d, causal != 0, deterministic, events,
+                     static_cast<cudaStream_t>(stream)));
 }
 }  // namespace
 
@@ -493,7 +525,8 @@ fa_status fa_fwd_standard(const void* q, const void* k, const void* v, void* o, 
 const char* fa_strerror(fa_status s) {
   switch (s) {
     case FA_OK: return "ok";
-    case FA_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size, bad scale or causal flag)";
+    case FA_ERR_INVALID_ARG:
+      return "invalid argument (null pointer, negative size, scale negative or not finite, bad causal flag)";
     case FA_ERR_UNSUPPORTED:
       return "unsupported shape (head dimension must be 64 or 128; e4m3 needs 128; decode takes at most 16 queries)";
     case FA_ERR_ALIGNMENT: return "misaligned pointer (tensors need 16-byte, lse 4-byte alignment)";
@@ -519,6 +552,8 @@ fa_status fa_device_status(void* stream, uint32_t* where) {
   if (where) *where = host[1];
   return host[0] == 0u ? FA_OK : FA_ERR_DEVICE_TIMEOUT;
 }
+
+fa_status fa_get_device_status(void* stream) { return fa_device_status(stream, nullptr); }
 
 fa_status fa_watchdog_selftest(uint32_t limit_us, void* stream) {
   if (limit_us == 0u || limit_us > 1000000u) return FA_ERR_INVALID_ARG;

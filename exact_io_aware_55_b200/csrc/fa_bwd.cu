@@ -626,7 +626,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool CAUSAL, bool DQ>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, cudaStream_t stream) {
+                         const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, void* const* events,
+                         cudaStream_t stream) {
+  // events (optional, cudaEvent_t[4]): recorded before launches 1, 2, 3 and after the last
+  auto mark = [&](int i) -> cudaError_t {
+    return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) : cudaSuccess;
+  };
+  cudaError_t e = mark(0);
+  if (e != cudaSuccess) return e;
   // 1) preprocess + zero the dQ accumulator
   constexpr int RPB = 256 / (D / 8);
   const long long rows = (long long)a.BH * a.Np;
@@ -634,7 +641,8 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   const long long dq_vec4 = DQ ? (long long)a.BH * a.N * D / 4 : 0;
   const int zero_blocks = DQ ? int(std::min<long long>((dq_vec4 + 255) / 256, 148LL * 8)) : 0;
   bwd_pre_kernel<D><<<row_blocks + zero_blocks, 256, 0, stream>>>(a, row_blocks, dq_vec4);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = mark(1);
   if (e != cudaSuccess) return e;
   // 2) main kernel
   constexpr size_t smem = bwd_smem_bytes<D>();
@@ -645,33 +653,38 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   const dim3 grid = CAUSAL ? dim3(unsigned(n_t) * unsigned(a.BH)) : dim3(n_t, a.BH);
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, tdq, a);
   e = cudaGetLastError();
+  if (e == cudaSuccess) e = mark(2);
   if (e != cudaSuccess) return e;
   if constexpr (!DQ) {
     // 3) deterministic dQ: query-tile-stationary pass, written once as bf16
-    return launch_bwd_dq<D, CAUSAL>(tq, tk, tv, tdo, a, stream);
+    e = launch_bwd_dq<D, CAUSAL>(tq, tk, tv, tdo, a, stream);
+  } else {
+    // 3) dQ -> bf16
+    const long long n8 = (long long)a.BH * a.N * D / 8;
+    const int fin_blocks = int(std::min<long long>((n8 + 255) / 256, 148LL * 8));
+    bwd_dq_final_kernel<<<fin_blocks, 256, 0, stream>>>(a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq), n8,
+                                                        a.scale);
+    e = cudaGetLastError();
   }
-  // 3) dQ -> bf16
-  const long long n8 = (long long)a.BH * a.N * D / 8;
-  const int fin_blocks = int(std::min<long long>((n8 + 255) / 256, 148LL * 8));
-  bwd_dq_final_kernel<<<fin_blocks, 256, 0, stream>>>(a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq), n8, a.scale);
-  return cudaGetLastError();
+  if (e == cudaSuccess) e = mark(3);
+  return e;
 }
 
 }  // namespace
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                        const CUtensorMap& tdq, const BwdArgs& a, int d, bool causal, bool deterministic,
-                       cudaStream_t stream) {
+                       void* const* events, cudaStream_t stream) {
   if (deterministic) {
-    if (d == 64) return causal ? launch_bwd_t<64, true, false>(tq, tk, tv, tdo, tdq, a, stream)
-                               : launch_bwd_t<64, false, false>(tq, tk, tv, tdo, tdq, a, stream);
-    return causal ? launch_bwd_t<128, true, false>(tq, tk, tv, tdo, tdq, a, stream)
-                  : launch_bwd_t<128, false, false>(tq, tk, tv, tdo, tdq, a, stream);
+    if (d == 64) return causal ? launch_bwd_t<64, true, false>(tq, tk, tv, tdo, tdq, a, events, stream)
+                               : launch_bwd_t<64, false, false>(tq, tk, tv, tdo, tdq, a, events, stream);
+    return causal ? launch_bwd_t<128, true, false>(tq, tk, tv, tdo, tdq, a, events, stream)
+                  : launch_bwd_t<128, false, false>(tq, tk, tv, tdo, tdq, a, events, stream);
   }
-  if (d == 64) return causal ? launch_bwd_t<64, true, true>(tq, tk, tv, tdo, tdq, a, stream)
-                             : launch_bwd_t<64, false, true>(tq, tk, tv, tdo, tdq, a, stream);
-  return causal ? launch_bwd_t<128, true, true>(tq, tk, tv, tdo, tdq, a, stream)
-                : launch_bwd_t<128, false, true>(tq, tk, tv, tdo, tdq, a, stream);
+  if (d == 64) return causal ? launch_bwd_t<64, true, true>(tq, tk, tv, tdo, tdq, a, events, stream)
+                             : launch_bwd_t<64, false, true>(tq, tk, tv, tdo, tdq, a, events, stream);
+  return causal ? launch_bwd_t<128, true, true>(tq, tk, tv, tdo, tdq, a, events, stream)
+                : launch_bwd_t<128, false, true>(tq, tk, tv, tdo, tdq, a, events, stream);
 }
 
 }  // namespace fa

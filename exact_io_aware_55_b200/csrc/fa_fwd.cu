@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float row_sum;
       if constexpr (!FP8) {
         uint32_t pk[64];
-        row_sum = need_mask ? row_exp128<false, 0>(sv, c, neg_m, pk)
+        row_sum = need_mask ? row_exp128<false, 0, true>(sv, c, neg_m, pk)
                             : row_exp128<false, S::kEmuPer8>(sv, c, neg_m, pk);
         uint32_t (&pa)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
         uint32_t (&pb)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_x32(s_tmem + 32, pb);
       } else {
         uint32_t pk[32];
-        row_sum = need_mask ? row_exp128<true, 0>(sv, c, neg_m, pk)
+        row_sum = need_mask ? row_exp128<true, 0, true>(sv, c, neg_m, pk)
                             : row_exp128<true, S::kEmuPer8>(sv, c, neg_m, pk);
         tmem_st_x32(s_tmem, pk);
       }

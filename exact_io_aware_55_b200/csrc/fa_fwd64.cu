@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
         uint32_t pk[64];
-        const float row_sum = need_mask ? row_exp128<false, 0>(sv, c, neg_m, pk)
+        const float row_sum = need_mask ? row_exp128<false, 0, true>(sv, c, neg_m, pk)
                                         : row_exp128<false, kEmuPer8>(sv, c, neg_m, pk);
         // P_g and O_g are free once O_g += P_g(j-1) V_(j-1) has completed (at
         // j = 0 the previous item's last product was awaited by its epilogue).

@@ -17,6 +17,7 @@
 // from different host threads without ordering) race on the array.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "fa.h"
@@ -31,16 +32,37 @@ constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices];
 
-// Device address of the scratch array on the current device.  The symbol's
-// name in host code is only a host-side stand-in; the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
-fa_status scratch_on_current_device(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_ARCH;
+// The current device must be an sm_100 part (the check fa_bwd makes too):
+// on any other GPU the kernels cannot run, and the symbol lookup below would
+// fail for the same reason.
+fa_status check_arch(int* dev_out) {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return FA_ERR_ARCH;
+  }
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FA_ERR_ARCH;
+  }
+  if (major != 10 || minor != 0) return FA_ERR_ARCH;
+  *dev_out = dev;
+  return FA_OK;
+}
+
+// Device address of the scratch array on device `dev` (the current one).  The
+// symbol's name in host code is only a host-side stand-in; the address comes
+// from cudaGetSymbolAddress, once per device, with that device current.  A
+// failed lookup leaves no pending error behind.
+fa_status scratch_on_device(int dev, void** out) {
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FA_ERR_LAUNCH;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return FA_ERR_ARCH;
+    }
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
@@ -56,6 +78,9 @@ size_t fa_bwd_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
                          int causal, void* stream) {
+  // Host-side argument checks first, so that a bad argument is reported as
+  // such whatever the shape's size.
+  if (!(std::isfinite(scale) && scale >= 0.0f) || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (need == static_cast<size_t>(-1)) {
     // Invalid shape: let fa_bwd report the precise code without touching the device.
@@ -63,9 +88,11 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   }
   if (need > kNoAllocScratchBytes) return FA_ERR_SCRATCH_LIMIT;
   if (need == 0) return fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, nullptr, 0, stream);
-  void* scratch = nullptr;
-  const fa_status st = scratch_on_current_device(&scratch);
+  int dev = 0;
+  fa_status st = check_arch(&dev);
   if (st != FA_OK) return st;
+  void* scratch = nullptr;
+  if ((st = scratch_on_device(dev, &scratch)) != FA_OK) return st;
   return fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, scratch, kNoAllocScratchBytes,
                 stream);
 }

@@ -37,13 +37,17 @@ __device__ __forceinline__ float row_max128(const float (&sv)[128]) {
 
 // p = 2^(s*c - m) for 128 scores; packs P for the PV MMA (bf16 pairs or e4m3
 // quads) and returns the fp32 row sum of p.  EMU of every 8 pairs (bf16) or
-// quads (e4m3) use the FMA-pipe exponential, the rest MUFU ex2.
-template <bool FP8, int EMU>
+// quads (e4m3) use the FMA-pipe exponential, the rest MUFU ex2.  MASKED rows
+// hold -inf for masked keys: with c = 0 (scale 0) the product -inf * 0 is NaN,
+// which max(x, -inf) turns back into -inf (max returns its non-NaN operand),
+// so a masked key still gets p = 0.
+template <bool FP8, int EMU, bool MASKED = false>
 __device__ __forceinline__ float row_exp128(const float (&sv)[128], float c, float neg_m,
                                             uint32_t (&pk)[FP8 ? 32 : 64]) {
   const float2 cc = make_float2(c, c), nm = make_float2(neg_m, neg_m);
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   auto ex = [&](float2 x, bool emu) {
+    if constexpr (MASKED) x = make_float2(fmaxf(x.x, -INFINITY), fmaxf(x.y, -INFINITY));
     return emu ? exp2_fma2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
   };
   if constexpr (!FP8) {

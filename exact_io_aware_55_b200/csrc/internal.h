@@ -158,9 +158,11 @@ cudaError_t launch_fwd64(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          bool causal, cudaStream_t stream);
 // tdq: map over the fp32 dQ accumulator (dims {d, N, BH}, box {32 columns,
 // 128 rows}); used by the d = 64 kernel's TMA bulk reductions.
+// events: optional cudaEvent_t[4] recorded on `stream` before the preprocess,
+// before the main kernel, after it, and after the last launch (NULL: none).
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdArgs& a, int d, bool causal,
-                       bool deterministic, cudaStream_t stream);
+                       bool deterministic, void* const* events, cudaStream_t stream);
 // Deterministic dQ pass (one 128-query tile per CTA, no atomics); defined in
 // fa_bwd_dq.cu, launched by launch_bwd after the dK/dV kernel.
 template <int D, bool CAUSAL>

@@ -25,7 +25,11 @@
  *     are masked.  B, H, N == 0 is a valid empty call that launches nothing.
  *   - causal != 0 selects top-left aligned causal masking (key j is visible to
  *     query i iff j <= i; Nq == Nk == N).  Fully masked tiles are skipped.
- *   - scale is the softmax scale (the configurations use 1/sqrt(d)).
+ *   - scale is the softmax scale (the configurations use 1/sqrt(d)).  It must
+ *     be finite and >= 0; scale = 0 is valid and makes every visible key
+ *     equally weighted (O is the mean of the visible V rows, LSE = ln of
+ *     their count, dQ = dK = 0).  A negative or non-finite scale returns
+ *     FA_ERR_INVALID_ARG.
  *   - stream is a cudaStream_t passed as an opaque pointer (NULL = legacy
  *     default stream).
  *   - Arguments are checked on the host before anything is launched; a bad
@@ -109,6 +113,23 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * fa_bwd with per-launch timing: the same computation, arguments and errors
+ * as fa_bwd, and additionally records four CUDA events (cudaEvent_t values
+ * passed as opaque pointers, created by the caller) on `stream`:
+ *   events[0] before the preprocess launch (D = rowsum(dO o O)),
+ *   events[1] before the recompute kernel (S, P, dV, dP, dS, dK, dQ),
+ *   events[2] after it, before the dQ conversion to bf16,
+ *   events[3] after the last launch.
+ * The elapsed time between events[1] and events[2] is the main kernel's own
+ * duration on the launching stream.  Any NULL event returns
+ * FA_ERR_INVALID_ARG before anything is launched.
+ */
+FA_API fa_status fa_bwd_events(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                               const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                               float scale, int causal, void* workspace, size_t workspace_bytes,
+                               void* const* events, void* stream);
+
+/*
  * Backward pass with a deterministic dQ: same arguments, outputs and workspace
  * as fa_bwd, but dQ is produced by a separate query-tile-parallel pass that
  * recomputes S, P and dP per query tile and accumulates dQ_i += dS K_j in
@@ -120,6 +141,21 @@ FA_API fa_status fa_bwd_deterministic(const void* q, const void* k, const void* 
                                       const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                                       float scale, int causal, void* workspace, size_t workspace_bytes,
                                       void* stream);
+
+/*
+ * Launch plan of fa_fwd and fa_fwd_fp8 for a shape, computed on the host as
+ * the forward computes it (no launch; uses the current device's SM count, or
+ * 148 when no device is visible).  A work item is one 128-row Q tile or a
+ * pair of them of one (batch, head):
+ *   *ctas       : CTAs launched (d = 64 non-causal runs at most one
+ *                 persistent CTA per SM over the items)
+ *   *items      : work items
+ *   *pair_items : items that hold a pair of Q tiles; on non-causal grids the
+ *                 pairs of a last round that would fill at most half of the
+ *                 SMs are split into single-tile items dispatched last.
+ * scale is not an argument; the other arguments are checked as in fa_fwd.
+ */
+FA_API fa_status fa_fwd_plan(int B, int H, int N, int d, int causal, int* ctas, int* items, int* pair_items);
 
 /*
  * Forward pass with float8 e4m3 inputs and per-tensor scales ("What changed
@@ -167,8 +203,8 @@ FA_API size_t fa_bwd_noalloc_max_bytes(void);
 
 /*
  * Decode against a KV cache: Nq (1..16) new queries per (batch, head) attend
- * over Nk cached keys ("It pairs naturally with the KV cache at inference",
- * chipfoundryservices glossary "flash attention").  The key range is split
+ * over Nk cached keys (chipfoundryservices glossary "flash attention", closing
+ * section: the method serves inference against a KV cache).  The key range is split
  * across CTAs; each split keeps its own running max and sum, and the splits
  * are combined by their log-sum-exp (O = sum_s exp(LSE_s - LSE) O_s).  HBM-
  * bound: K and V are read once.
@@ -222,6 +258,12 @@ FA_API const char* fa_strerror(fa_status status);
  * not NULL, receives a code naming the wait that gave up.
  */
 FA_API fa_status fa_device_status(void* stream, uint32_t* where);
+
+/*
+ * fa_device_status(stream, NULL): the device status check without the code
+ * of the wait site.
+ */
+FA_API fa_status fa_get_device_status(void* stream);
 
 /*
  * Self-test of the bounded-wait machinery: launches one block that waits on a

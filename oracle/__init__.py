@@ -33,7 +33,8 @@ Pins (see tests/test_oracle_pins.py): brute-force triple loops, an independent
 online-softmax recurrence, closed forms (constant scores -> mean of V, N = 1),
 convex hull / affine / permutation invariants, central finite differences of
 L = sum(dO o O), and the gradient sum identities.  No function here is
-"parity unpinned".
+"parity unpinned": the rectangular (decode) functions are pinned in
+tests/test_oracle_decode.py.
 """
 from __future__ import annotations
 
@@ -183,9 +184,10 @@ def head_backward_sampled(qh, kh, vh, doh, scale, causal, rows, cols):
 
 
 def head_forward_rect(qh, kh, vh, scale, causal):
-    """Forward of one head with Nq query rows against Nk keys (decode against a
-    KV cache: explainers' glossary page, "It pairs naturally with the KV cache at
-    inference").  Causal masking is aligned to the end of the key sequence:
+    """Forward of one head with Nq query rows against Nk keys: decoding new
+    queries against a KV cache (chipfoundryservices glossary "flash attention",
+    closing section, which names inference with a KV cache as the setting the
+    method is used in).  Causal masking is aligned to the end of the key sequence:
     query i (0-based among the Nq) sees keys j <= Nk - Nq + i, so the Nq queries
     are the last Nq positions of a causal sequence of length Nk.  Plain
     definition, full rows, two-pass softmax.  Returns (O [Nq, d], LSE [Nq])."""

@@ -21,7 +21,9 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
-    assert {"fa_fwd", "fa_bwd", "fa_fwd_fp8", "fa_bwd_workspace_size", "fa_strerror"} <= set(names)
+    # the boundary's method calls, named as the hot-path scope lists them
+    assert {"fa_fwd", "fa_bwd", "fa_fwd_fp8", "fa_bwd_workspace_size", "fa_strerror",
+            "fa_get_device_status"} <= set(names)
     lib = ctypes.CDLL(fa.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -56,7 +58,8 @@ def fwd(q, o, lse, B=1, H=1, N=128, d=64, scale=0.125, causal=0):
 def test_forward_argument_errors_launch_nothing():
     assert fwd(None, None, None) == C["FA_ERR_INVALID_ARG"]
     assert fwd(4096, 4096, 4096, d=96) == C["FA_ERR_UNSUPPORTED"]
-    assert fwd(4096, 4096, 4096, scale=0.0) == C["FA_ERR_INVALID_ARG"]
+    assert fwd(4096, 4096, 4096, scale=-0.125) == C["FA_ERR_INVALID_ARG"]
+    assert fwd(4096, 4096, 4096, scale=float("inf")) == C["FA_ERR_INVALID_ARG"]
     assert fwd(4096, 4096, 4096, scale=float("nan")) == C["FA_ERR_INVALID_ARG"]
     assert fwd(4096, 4096, 4096, causal=2) == C["FA_ERR_INVALID_ARG"]
     assert fwd(4096, 4096, 4096, N=-5) == C["FA_ERR_INVALID_ARG"]
@@ -167,3 +170,40 @@ def test_standard_workspace_and_errors():
     assert std(q=p + 8) == C["FA_ERR_ALIGNMENT"]
     assert std(d=96) == C["FA_ERR_UNSUPPORTED"]
     assert std(q=None) == C["FA_ERR_INVALID_ARG"]
+
+
+def test_scale_zero_passes_the_argument_checks():
+    # scale = 0 is a valid (uniform-weight) softmax: the call gets past every
+    # host check and stops only at the device query on a host without a GPU
+    st = fwd(4096, 4096, 4096, scale=0.0)
+    assert st in (C["FA_ERR_ARCH"], C["FA_OK"], C["FA_ERR_LAUNCH"])
+    assert st != C["FA_ERR_INVALID_ARG"]
+
+
+def test_forward_plan_on_the_mixed_grid():
+    """B4 H16 N2048 d128 non-causal: 512 Q-tile pairs on 148 SMs leave a last
+    round of 68, which is split into 136 single-tile items dispatched last."""
+    if fa.lib.fa_get_device_status(None) != C["FA_ERR_ARCH"]:
+        pytest.skip("a GPU is visible; the GPU test checks the plan with its SM count")
+    assert fa.fa_fwd_plan(4, 16, 2048, 128, False) == (580, 580, 444)
+    assert fa.fa_fwd_plan(4, 16, 2048, 64, False) == (148, 580, 444)     # persistent CTAs
+    assert fa.fa_fwd_plan(4, 16, 2048, 128, True) == (512, 512, 512)     # causal: pairs only
+    assert fa.fa_fwd_plan(1, 32, 8192, 128, False) == (1024, 1024, 1024)  # 1024 = 148 * 6 + 136: no split
+    assert fa.fa_fwd_plan(1, 1, 0, 128, False) == (0, 0, 0)
+    with pytest.raises(fa.FAError):
+        fa.fa_fwd_plan(1, 1, 16, 96, False)
+
+
+def test_bwd_events_needs_four_events():
+    p = 4096
+    args = [p] * 9
+    need = fa.fa_bwd_workspace_size(1, 1, 64, 64)
+    assert fa.lib.fa_bwd_events(*args, 1, 1, 64, 64, F(0.125), 0, p, need, None, None) == C["FA_ERR_INVALID_ARG"]
+    ev = (ctypes.c_void_p * 4)(p, p, None, p)
+    assert fa.lib.fa_bwd_events(*args, 1, 1, 64, 64, F(0.125), 0, p, need, ev, None) == C["FA_ERR_INVALID_ARG"]
+
+
+def test_get_device_status_without_a_gpu():
+    if fa.lib.fa_get_device_status(None) == C["FA_OK"]:
+        pytest.skip("a GPU is visible")
+    assert fa.lib.fa_get_device_status(None) == C["FA_ERR_ARCH"]

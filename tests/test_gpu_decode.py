@@ -98,3 +98,12 @@ def test_decode_workload_b8_h32_nk16384_d128_sampled(causal):
         qh, kh, vh = (synth.head_f64(inp, n, b, h) for n in ("q", "k", "v"))
         o_ref, lse_ref = oracle.head_forward_rect(qh, kh, vh, d ** -0.5, causal)
         gu.assert_o_lse(o[b, h], lse[b, h], o_ref, lse_ref, f"head {(b, h)}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_decode_scale_zero(causal):
+    """scale = 0 over several splits: uniform weights over the visible keys."""
+    inp = synth.decode_inputs(1, 2, 3, 5000, 128, seed=93)
+    o, lse, scale = _run(inp, causal, scale=0.0)
+    o_ref, lse_ref = oracle.attention_forward_rect(inp["q"], inp["k"], inp["v"], 0.0, causal)
+    gu.assert_o_lse(o, lse, o_ref, lse_ref, f"scale 0 causal={causal}")

@@ -67,3 +67,27 @@ def test_fp8_rejects_d64():
     with pytest.raises(fa.FAError) as e:
         fa.attention_forward_fp8(x, x, x, 1.0, 1.0, 1.0)
     assert e.value.status == fa.STATUS_CODES["FA_ERR_UNSUPPORTED"]
+
+
+def test_fp8_mixed_pair_single_grid_b4_h16_n2048_d128():
+    """The e4m3 forward on the mixed grid (444 pair blocks, then 136 single
+    Q-tile blocks on 148 SMs): every head in full against the oracle."""
+    B, H, N, d = 4, 16, 2048, 128
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert fa.fa_fwd_plan(B, H, N, d, False) == (580, 580, 444)
+    inp = synth.attention_inputs(B, H, N, d, seed=1246, storage="e4m3")
+    o, lse, scale = _run(inp, False)
+    o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], scale, False)
+    _check(o, lse, o_ref, lse_ref, "mixed grid")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_scale_zero_gives_the_mean_of_v(causal):
+    B, H, N, d = 1, 2, 300, 128
+    inp = synth.attention_inputs(B, H, N, d, seed=1247, storage="e4m3")
+    q8, k8, v8 = (gu.dev_u8(inp[n + "_bits"]) for n in ("q", "k", "v"))
+    o, lse = fa.attention_forward_fp8(q8, k8, v8, inp["q_descale"], inp["k_descale"], inp["v_descale"],
+                                      scale=0.0, causal=causal)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], 0.0, causal)
+    _check(gu.to_f64(o), gu.to_f64(lse), o_ref, lse_ref, f"scale 0 causal={causal}")

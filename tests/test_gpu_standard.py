@@ -16,9 +16,9 @@ pytestmark = pytest.mark.gpu
 fa = pytest.importorskip("exact_io_aware_55_b200")
 
 
-def _run(inp, causal):
+def _run(inp, causal, scale=None):
     B, H, N, d = inp["shape"]
-    scale = 1.0 / math.sqrt(d)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
     q, k, v = (gu.dev_bf16(inp[n + "_bits"]) for n in ("q", "k", "v"))
     og = gu.Guarded((B, H, N, d), torch.bfloat16)
     lg = gu.Guarded((B, H, N), torch.float32)
@@ -55,3 +55,11 @@ def test_standard_matches_fused_b4_h16_n2048_d64(causal):
         qh, kh, vh = (synth.head_f64(inp, n, b, h) for n in ("q", "k", "v"))
         o_ref, lse_ref = oracle.head_forward(qh, kh, vh, scale, causal, rows=rows)
         gu.assert_o_lse(o[b, h, rows], lse[b, h, rows], o_ref, lse_ref, f"head {(b, h)}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_standard_scale_zero(causal):
+    inp = synth.attention_inputs(1, 2, 300, 64, seed=1248, with_grad=False)
+    o, lse, _, _ = _run(inp, causal, scale=0.0)
+    o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], 0.0, causal)
+    gu.assert_o_lse(o, lse, o_ref, lse_ref, f"scale 0 causal={causal}")

@@ -5,8 +5,9 @@ allocation, or a serving loop that reserves all its memory at start-up and
 must not call cudaMalloc afterwards -- get the same backward with no caller
 workspace: the scratch is a fixed array inside the library.  These tests call
 the entry point through the C ABI (raw pointers via ctypes) and check, on two
-calls in a row, that it returns what fa_bwd returns with a caller workspace,
-within the gradient tolerance the parity tests use.  The file is named to be
+calls in a row, that it returns what fa_bwd returns with a caller workspace:
+dK and dV byte for byte, dQ (fp32 atomics) within the gradient tolerance the
+parity tests use.  The file is named to be
 collected last.
 """
 import ctypes
@@ -35,25 +36,55 @@ def _call_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale, causal):
                                  B, H, N, d, ctypes.c_float(scale), int(causal), stream)
 
 
-@pytest.mark.parametrize("shape,causal", [((2, 4, 1000, 64), False), ((1, 3, 777, 128), True)])
-def test_noalloc_matches_fa_bwd_on_two_calls(shape, causal):
+def _case(shape, causal, seed):
     B, H, N, d = shape
     assert fa.fa_bwd_workspace_size(B, H, N, d) <= fa.lib.fa_bwd_noalloc_max_bytes()
-    inp = synth.attention_inputs(B, H, N, d, seed=900 + N, want_f64=False)
+    inp = synth.attention_inputs(B, H, N, d, seed=seed, want_f64=False)
     q, k, v, do = (gu.dev_bf16(inp[n + "_bits"]) for n in ("q", "k", "v", "do"))
     scale = 1.0 / math.sqrt(d)
     o, lse = fa.attention_forward(q, k, v, scale=scale, causal=causal)
-    ref = [gu.to_f64(t) for t in fa.attention_backward(q, k, v, o, do, lse, scale=scale, causal=causal)]
+    ref = fa.attention_backward(q, k, v, o, do, lse, scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    return (q, k, v, o, do, lse, scale, causal), ref
+
+
+def _check(args, ref):
+    q = args[0]
+    outs = [torch.full_like(q, float("nan")) for _ in range(3)]
+    st = _call_noalloc(*args[:6], *outs, args[6], args[7])
+    assert st == 0, fa.strerror(st)
+    torch.cuda.synchronize()
+    # dQ goes through fp32 atomics in both calls: equal within the gradient tolerance
+    g, r = gu.to_f64(outs[0]), gu.to_f64(ref[0])
+    assert np.all(np.isfinite(g)) and gu.rel_fro(g, r) <= gu.GRAD_REL_FRO, "dQ"
+    # dK and dV are summed in a fixed order on chip: identical bytes, so any
+    # stale scratch content (row statistics of an earlier call) would show
+    for name, got, want in zip(("dK", "dV"), outs[1:], ref[1:]):
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), name
+
+
+def test_noalloc_matches_fa_bwd_on_two_calls_larger_then_smaller():
+    """A shape that fills most of the scratch, then smaller ones (one causal,
+    one with a ragged last tile) right after it, each twice: every call must
+    equal fa_bwd with a caller workspace on the same inputs."""
+    big = _case((2, 8, 7600, 128), False, 901)      # 60.3 MiB of the 64 MiB scratch
+    small = [_case((2, 4, 1000, 64), False, 902), _case((1, 3, 777, 128), True, 903)]
     for _ in range(2):
-        outs = [torch.full_like(q, float("nan")) for _ in range(3)]
-        st = _call_noalloc(q, k, v, o, do, lse, *outs, scale, causal)
-        assert st == 0, fa.strerror(st)
-        torch.cuda.synchronize()
-        for name, got, r in zip(("dQ", "dK", "dV"), outs, ref):
-            g = gu.to_f64(got)
-            assert np.all(np.isfinite(g)), name
-            assert gu.rel_fro(g, r) <= gu.GRAD_REL_FRO, name
+        _check(*big)
+        for c in small:
+            _check(*c)
     assert fa.fa_device_status() == (0, 0)
+
+
+def test_noalloc_checks_arguments_before_the_size_limit():
+    B, H, N, d = 1, 32, 4096, 128
+    assert fa.fa_bwd_workspace_size(B, H, N, d) > fa.lib.fa_bwd_noalloc_max_bytes()
+    x = torch.empty((B, H, N, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    outs = [torch.empty_like(x) for _ in range(3)]
+    for scale, causal in ((float("nan"), False), (-1.0, False), (0.125, 2)):
+        st = _call_noalloc(x, x, x, x, x, lse, *outs, scale, causal)
+        assert st == fa.STATUS_CODES["FA_ERR_INVALID_ARG"], (scale, causal, st)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
