@@ -4,14 +4,20 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one pass of the whole bf16 path over one batch: fa_fwd (O, LSE)
-followed by fa_bwd (preprocess, recompute kernel, dQ finalize).  The workload
-is the B=4, H=16, N=2048, d=64 non-causal bf16 attention with Q, K, V, dO ~
-N(0, 1) (seeded synthetic inputs).  The metric is attention TFLOP/s:
+followed by fa_bwd (preprocess, recompute kernel, dQ conversion).  The
+workload is the long-context causal attention B=1, H=32, N=32768, d=128 with
+Q, K, V, dO ~ N(0, 1) (seeded synthetic inputs): the largest of the attention
+configurations, and it fits one GPU.  The metric is attention TFLOP/s:
   forward FLOPs F = 4 B H N^2 d (halved when causal), backward 2.5 F,
   fwd+bwd TFLOP/s = 3.5 F / (t_fwd + t_bwd).
-Rank 0 prints ONE JSON line.  Under torchrun every rank runs its own batch
-(weak scaling, no collective on the data path); `value` is the FLOPs of all
-ranks divided by the slowest rank's time.
+Rank 0 prints ONE JSON line.
+
+With --gpus N > 1 outside a torchrun environment the script re-launches itself
+under torch.distributed.run with N ranks (one per GPU).  The B*H heads of the
+one problem are split into contiguous slices, one per rank: heads are
+independent, so there is no collective on the data path (NCCL only takes the
+max of the ranks' times).  `value` is the whole problem's FLOPs divided by the
+slowest rank's time: the total work is fixed as N grows (strong scaling).
 
 `--impl reference` times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of the same workload on the host cores.
@@ -33,8 +39,10 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = dict(B=4, H=16, N=2048, d=64, causal=False)
-WORKLOAD_NAME = "attention fwd+bwd bf16 B4 H16 N2048 d64 non-causal"
+WORKLOAD = dict(B=1, H=32, N=32768, d=128, causal=True)
+WORKLOAD_NAME = "attention fwd+bwd bf16 B1 H32 N32768 d128 causal"
+WORKLOAD_SEED = 1238                 # the seed of this configuration's parity test
+CPU_SAMPLE_N = 4096                  # rows and keys of the CPU oracle's sample unit
 METRIC = "attention TFLOP/s fwd & fwd+bwd (bf16) and % of B200 dense tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
@@ -113,17 +121,43 @@ class ClockSampler:
 
 # -------------------------------------------------------------- our arm
 def apply_shape(args):
-    """--shape/--causal select another workload (profiling runs); the default
-    is the bench workload."""
+    """--shape/--causal/--noncausal select another workload (profiling runs);
+    the default is the bench workload."""
     global WORKLOAD_NAME
     if args.shape:
         B, H, N, d = (int(x) for x in args.shape.split(","))
         WORKLOAD.update(B=B, H=H, N=N, d=d)
     if args.causal:
         WORKLOAD["causal"] = True
-    if args.shape or args.causal:
+    if args.noncausal:
+        WORKLOAD["causal"] = False
+    if args.shape or args.causal or args.noncausal:
         WORKLOAD_NAME = (f"attention fwd+bwd bf16 B{WORKLOAD['B']} H{WORKLOAD['H']} N{WORKLOAD['N']} "
                          f"d{WORKLOAD['d']} {'causal' if WORKLOAD['causal'] else 'non-causal'}")
+
+
+def spawn_ranks(args) -> int:
+    """Re-launch this script under torch.distributed.run with one rank per GPU."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def rank_heads(B, H, ws, rank):
+    """This rank's contiguous slice [h0, h1) of the flattened B*H heads."""
+    from exact_io_aware_55_b200.dist import head_range
+    return head_range(B * H, ws, rank)
+
+
+def head_slice(bits, B, H, h0, h1):
+    """Heads [h0, h1) of a [B, H, N, d] array as a contiguous [1, h1-h0, N, d]
+    array (a [B, H, N, d] tensor is B*H consecutive heads)."""
+    N, d = bits.shape[2], bits.shape[3]
+    return np.ascontiguousarray(bits.reshape(B * H, N, d)[h0:h1]).reshape(1, h1 - h0, N, d)
 
 
 def run_ours(args):
@@ -140,23 +174,24 @@ def run_ours(args):
         import datetime
 
         import torch.distributed as dist
-        # long enough for rank 0's extra measurements while the others wait at the last barrier
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     dev = torch.device("cuda", local)
     B, H, N, d, causal = (WORKLOAD[k] for k in ("B", "H", "N", "d", "causal"))
+    h0, h1 = rank_heads(B, H, ws, rank)
+    nh = h1 - h0
     scale = 1.0 / math.sqrt(d)
-    seed = 4242 + rank
-    inp = synth.attention_inputs(B, H, N, d, seed=seed, want_f64=False)
+    inp = synth.attention_inputs(B, H, N, d, seed=WORKLOAD_SEED, want_f64=False)
+    host_in = {n: head_slice(inp[n + "_bits"], B, H, h0, h1) for n in ("q", "k", "v", "do")}
+    del inp
 
     def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
 
-    q, k, v, do = (to_dev(inp[n + "_bits"]) for n in ("q", "k", "v", "do"))
+    q, k, v, do = (to_dev(host_in[n]) for n in ("q", "k", "v", "do"))
     o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    lse = torch.empty((1, nh, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    wsz = fa.fa_bwd_workspace_size(B, H, N, d)
-    work = torch.empty(wsz, dtype=torch.uint8, device=dev)
+    work = torch.empty(max(16, fa.fa_bwd_workspace_size(1, nh, N, d)), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -164,7 +199,8 @@ def run_ours(args):
         fa.fa_fwd(q, k, v, o, lse, scale, causal, stream)
         fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale, causal, work, stream)
 
-    F = fwd_flops(B, H, N, d, causal)
+    F_all = fwd_flops(B, H, N, d, causal)          # the whole problem, all ranks
+    F_rank = fwd_flops(1, nh, N, d, causal)        # this rank's slice
 
     def timed(K, W, sampler_window_s=args.clock_window):
         for _ in range(W):
@@ -176,12 +212,12 @@ def run_ours(args):
         sampler.start()
         t_end = time.time() + sampler_window_s
         while time.time() < t_end:
-            for _ in range(20):
+            for _ in range(5):
                 flush.fill_(1.0)
                 step()
             torch.cuda.synchronize()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-               torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        # per step: [start, fwd done = bwd start, main kernel start, main kernel end, bwd end]
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize()
@@ -189,18 +225,16 @@ def run_ours(args):
             flush.fill_(1.0)                     # L2 flush, outside the events
             ev[i][0].record(stream)
             fa.fa_fwd(q, k, v, o, lse, scale, causal, stream)
-            ev[i][1].record(stream)
-            fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, scale, causal, work, stream)
-            ev[i][2].record(stream)
+            fa.fa_bwd_events(q, k, v, o, do, lse, dq, dk, dv, scale, causal, work, ev[i][1:], stream)
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
         clocks = sampler.stop()
-        t_fwd = sum(a.elapsed_time(b) for a, b, _ in ev) / K
-        t_bwd = sum(b.elapsed_time(c) for _, b, c in ev) / K
-        return t_fwd, t_bwd, clocks
+        mean = lambda a, b: sum(e[a].elapsed_time(e[b]) for e in ev) / K  # noqa: E731
+        return {"fwd": mean(0, 1), "bwd": mean(1, 4), "pre": mean(1, 2), "main": mean(2, 3),
+                "fin": mean(3, 4)}, clocks
 
-    t_fwd, t_bwd, clocks = timed(args.steps, args.warmup)
+    t, clocks = timed(args.steps, args.warmup)
     # Re-measure once if any rank saw a throttle reason; the decision is taken
     # together so that every rank runs the same collectives.
     bad = any(r in clocks["reasons"] for r in BAD_REASONS)
@@ -209,24 +243,25 @@ def run_ours(args):
         dist.all_reduce(flag, op=dist.ReduceOp.MAX)
         bad = flag.item() > 0.0
     if bad:
-        t_fwd, t_bwd, clocks = timed(args.steps, args.warmup)
+        t, clocks = timed(args.steps, args.warmup)
         clocks["remeasured"] = True
     st, where = fa.fa_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status {st} (wait site {where}) during the bench")
 
-    t_step, t_fwd, t_bwd = max_over_ranks(dist, [t_fwd + t_bwd, t_fwd, t_bwd], dev)
-    value = ws * 3.5 * F / (t_step * 1e-3) / 1e12
-    fwd_tflops = ws * F / (t_fwd * 1e-3) / 1e12
-    bwd_tflops = ws * 2.5 * F / (t_bwd * 1e-3) / 1e12
+    t_step, t_fwd, t_bwd, t_main, t_pre, t_fin = max_over_ranks(
+        dist, [t["fwd"] + t["bwd"], t["fwd"], t["bwd"], t["main"], t["pre"], t["fin"]], dev)
+    value = 3.5 * F_all / (t_step * 1e-3) / 1e12
+    fwd_tflops = F_all / (t_fwd * 1e-3) / 1e12
+    bwd_tflops = 2.5 * F_all / (t_bwd * 1e-3) / 1e12
 
     # ---------------- e2e through the public API with pinned host buffers
     # Every step copies its inputs host -> device, runs fa_fwd + fa_bwd and
     # copies O, LSE, dQ, dK, dV back.  Three streams (H2D, compute, D2H) and
     # two device buffer sets let step i's upload and step i-1's download
     # overlap with the kernels; events order each buffer's reuse.
-    host = {n: torch.from_numpy(np.ascontiguousarray(inp[n + "_bits"]).view(np.int16)).view(torch.bfloat16)
-            .pin_memory() for n in ("q", "k", "v", "do")}
+    host = {n: torch.from_numpy(host_in[n].view(np.int16)).view(torch.bfloat16).pin_memory()
+            for n in ("q", "k", "v", "do")}
     out_names = ("o", "lse", "dq", "dk", "dv")
     shapes = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
     host_out = [{n: torch.empty(shapes[n].shape, dtype=shapes[n].dtype, pin_memory=True) for n in out_names}
@@ -234,8 +269,8 @@ def run_ours(args):
     dev_in = [{n: torch.empty_like(host[n], device=dev) for n in host} for _ in range(2)]
     dev_out = [{n: torch.empty_like(shapes[n]) for n in out_names} for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev = lambda: torch.cuda.Event()  # noqa: E731
-    in_ready, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    mk = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, comp_done, out_done = [mk(), mk()], [mk(), mk()], [mk(), mk()]
     started = [False, False]
 
     def e2e_step(i):
@@ -264,7 +299,7 @@ def run_ours(args):
     for i in range(3):
         e2e_step(i)
     torch.cuda.synchronize()
-    K2 = max(5, min(args.steps, 50))
+    K2 = max(5, min(args.steps, 30))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
@@ -277,41 +312,59 @@ def run_ours(args):
     e1.record(s_out)
     torch.cuda.synchronize()
     t_e2e = max_over_ranks(dist, [e0.elapsed_time(e1) / K2], dev)[0]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    d2h = sum(x.numel() * x.element_size() for x in host_out[0].values())
+    del host, host_out, dev_in, dev_out
 
-    # ---------------- extra measurements (rank 0, not part of `value`)
+    # ---------------- extra measurements (rank 0 of a 1-GPU run, not part of `value`)
     extra = {}
-    if rank == 0 and not args.no_extra:
-        extra = extra_measurements(fa, torch, synth, dev, stream)
+    if rank == 0 and ws == 1 and not args.no_extra:
+        del q, k, v, do, o, lse, dq, dk, dv, work
+        torch.cuda.empty_cache()
+        extra = extra_measurements(fa, torch, dev, stream, flush)
 
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    roof = {"bound": "tensor", "kernel": "fa_bwd (bwd_kernel + its preprocess and dQ-finalize launches)",
-            "achieved": round(bwd_tflops / ws, 2), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(bwd_tflops / ws / peak, 4), "traffic": committed_traffic("bwd_kernel", WORKLOAD_NAME),
-            "peak_source": f"{peak_src} bf16_tflops (burst; each launch is timed alone)"}
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
+    # the dominant kernel: the backward's recompute kernel, 2.5 F of this rank's slice per launch
+    main_tflops = 2.5 * F_rank / (t_main * 1e-3) / 1e12 if nh else 0.0
+    call_tflops = 2.5 * F_rank / (t_bwd * 1e-3) / 1e12 if nh else 0.0
+    roof = {"bound": "tensor", "kernel": "bwd_kernel<128, causal> (the backward's recompute kernel)",
+            "achieved": round(main_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(main_tflops / peak, 4),
+            "traffic": committed_traffic("bwd_kernel", WORKLOAD_NAME) if ws == 1 else None,
+            "algorithmic_flops_per_launch": 2.5 * F_rank,
+            "ms_per_launch": round(t_main, 5),
+            "peak_source": f"{peak_src} bf16_tflops (burst)",
+            "frac_of_sustained_peak": round(main_tflops / peak_sus, 4),
+            "fa_bwd_call": {"achieved": round(call_tflops, 2), "frac": round(call_tflops / peak, 4),
+                            "ms": round(t_bwd, 5), "ms_preprocess": round(t_pre, 5),
+                            "ms_dq_convert": round(t_fin, 5)}}
 
     if rank == 0:
         cpu = cpu_baseline(args) if (ws == 1 and not args.no_cpu_baseline) else None
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Philox, rounded to bf16)",
+            "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) Philox, rounded to bf16)",
             "config": {"workload": WORKLOAD_NAME, "B": B, "H": H, "N": N, "d": d, "causal": causal,
-                       "global_batch": B * ws, "seq_len": N, "parallelism": f"dp{ws} (independent batches)",
-                       "l2": "256 MiB flush write between steps, outside the per-step CUDA events"},
+                       "seed": WORKLOAD_SEED, "global_batch": B, "seq_len": N,
+                       "parallelism": f"heads split over {ws} GPU(s), {nh} on rank 0, no data-path collective",
+                       "l2": "inputs (4 x 256 MiB per GPU at one GPU) exceed L2; plus a 256 MiB flush write "
+                             "between steps, outside the per-step CUDA events"},
             "fwd_tflops": round(fwd_tflops, 2), "bwd_tflops": round(bwd_tflops, 2),
             "fwd_frac_of_peak": round(fwd_tflops / ws / peak, 4),
+            "bwd_frac_of_peak": round(bwd_tflops / ws / peak, 4),
             "fwd_bwd_frac_of_peak": round(value / ws / peak, 4),
             "ms_fwd": round(t_fwd, 5), "ms_bwd": round(t_bwd, 5),
-            "e2e": {"value": round(ws * 3.5 * F / (t_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-                    "ms_per_step": round(t_e2e, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "e2e": {"value": round(3.5 * F_all / (t_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "ms_per_step": round(t_e2e, 4), "h2d_bytes_per_step": h2d * ws, "d2h_bytes_per_step": d2h * ws,
                     "api": "fa_fwd + fa_bwd on pinned-host inputs copied in and results copied out every "
                            "step; copy and compute streams overlap neighbouring steps"},
             "gpu_launches": 4 * args.steps,
             "roofline": roof,
-            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
+            "clocks": {k_: clocks[k_] for k_ in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
             "cpu_baseline": cpu,
             "extra": extra,
         }
@@ -323,8 +376,9 @@ def run_ours(args):
 
 def run_case(args):
     """One named path on --shape, for profiling (a short JSON line, not the
-    bench line): 'decode' (B,H,Nk,d with --nq queries, causal) or 'standard'
-    (B,H,N,d: the materialising baseline, then the fused forward, per step)."""
+    bench line): 'decode' (B,H,Nk,d with --nq queries, causal), 'standard'
+    (B,H,N,d: the materialising baseline, then the fused forward, per step) or
+    'fp8' (B,H,N,d: the e4m3 forward)."""
     import torch
 
     import exact_io_aware_55_b200 as fa
@@ -339,6 +393,7 @@ def run_case(args):
     def rnd(*shape):
         return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
 
+    nbytes, flops = None, None
     if args.case == "decode":
         q, k, v = rnd(B, H, args.nq, d), rnd(B, H, N, d), rnd(B, H, N, d)
         o = torch.empty_like(q)
@@ -349,6 +404,15 @@ def run_case(args):
         def step():
             fa.fa_fwd_decode(q, k, v, o, lse, d ** -0.5, True, work, stream)
         nbytes = 4 * B * H * N * d
+    elif args.case == "fp8":
+        q8, k8, v8 = (torch.randn((B, H, N, d), generator=g, device=dev).mul_(100.0).clamp_(-448, 448)
+                      .to(torch.float8_e4m3fn) for _ in range(3))
+        o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, H, N), device=dev)
+
+        def step():
+            fa.fa_fwd_fp8(q8, k8, v8, 0.01, 0.01, 0.01, o, lse, d ** -0.5, args.causal, stream)
+        flops = fwd_flops(B, H, N, d, args.causal)
     else:
         q, k, v = rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d)
         o = torch.empty_like(q)
@@ -358,7 +422,6 @@ def run_case(args):
         def step():
             fa.fa_fwd_standard(q, k, v, o, lse, d ** -0.5, args.causal, work, stream)
             fa.fa_fwd(q, k, v, o, lse, d ** -0.5, args.causal, stream)
-        nbytes = None
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -372,10 +435,12 @@ def run_case(args):
     if st != 0:
         raise RuntimeError(f"device status {st} (wait site {where})")
     ms = e0.elapsed_time(e1) / args.steps
-    line = {"case": args.case, "shape": args.shape, "ms_per_step": round(ms, 5)}
+    line = {"case": args.case, "shape": args.shape, "causal": bool(args.causal), "ms_per_step": round(ms, 5)}
     if nbytes:
         line["nq"] = args.nq
         line["gbs"] = round(nbytes / ms / 1e6, 1)
+    if flops:
+        line["tflops"] = round(flops / ms / 1e9, 1)
     print(json.dumps(line), flush=True)
 
 
@@ -413,84 +478,82 @@ def committed_traffic(kernel: str, workload: str):
     return None
 
 
-def extra_measurements(fa, torch, synth, dev, stream):
-    """Single-GPU context numbers: long-sequence non-causal bf16 (fwd and bwd at
-    N=8192, d=128), the causal B2 H16 N8192 and B1 H32 N32768 d128
-    configurations, the e4m3 forward at B2 H16 N16384 d128, standard
-    (materialising) attention against the fused forward, and the split-KV
-    decode (1 and 4 queries over a 16384-key cache, 8 x 32 heads, d=128)."""
+def extra_measurements(fa, torch, dev, stream, flush):
+    """Single-GPU context numbers, each call timed with CUDA events on the
+    launching stream with the L2 flush write between calls: the B4 H16 N2048
+    d64 non-causal configuration, long-sequence non-causal bf16 (N=8192,
+    d=128), the causal B2 H16 N8192 d128 configuration, the e4m3 forward at B2
+    H16 N16384 d128, standard (materialising) attention against the fused
+    forward, and the split-KV decode (1 and 4 queries over a 16384-key cache,
+    8 x 32 heads, d=128)."""
     out = {}
 
-    def time_call(fn, iters=10, warm=3):
-        for _ in range(warm):
-            fn()
+    def time_call(fn, iters=10, warm=3, parts=False):
+        """Mean ms per call; with parts=True fn takes four events (fa_bwd_events)
+        and the result also holds the main kernel's own time."""
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(iters)]
+        for i in range(warm):
+            flush.fill_(1.0)
+            fn(evs[0][1:]) if parts else fn()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(iters):
-            fn()
-        e1.record(stream)
+        for i in range(iters):
+            flush.fill_(1.0)
+            evs[i][0].record(stream)
+            if parts:
+                fn(evs[i][1:])
+            else:
+                fn()
+                evs[i][4].record(stream)
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / iters
+        ms = sum(e[0].elapsed_time(e[4]) for e in evs) / iters
+        if not parts:
+            return ms
+        return ms, sum(e[2].elapsed_time(e[3]) for e in evs) / iters
 
     peaks, _ = load_peaks()
-    B, H, N, d = 1, 32, 8192, 128
+    pk = peaks["bf16_tflops"]
     g = torch.Generator(device=dev)
     g.manual_seed(7)
-    q, k, v, do = (torch.randn((B, H, N, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-                   for _ in range(4))
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    work = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
-    sc = 1.0 / math.sqrt(d)
-    F = fwd_flops(B, H, N, d, False)
-    tf = time_call(lambda: fa.fa_fwd(q, k, v, o, lse, sc, False, stream))
-    tb = time_call(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, sc, False, work, stream))
-    out["noncausal_b1_h32_n8192_d128"] = {
-        "fwd_tflops": round(F / tf / 1e9, 1), "fwd_frac": round(F / tf / 1e9 / peaks["bf16_tflops"], 4),
-        "bwd_tflops": round(2.5 * F / tb / 1e9, 1), "bwd_frac": round(2.5 * F / tb / 1e9 / peaks["bf16_tflops"], 4),
-        "inputs": "N(0,1) from torch's seeded CUDA generator (timing only)"}
-    del q, k, v, do, o, dq, dk, dv, work
-    # the named causal configurations: B2 H16 N8192 d128 and B1 H32 N32768 d128
-    for (B, H, N, d) in ((2, 16, 8192, 128), (1, 32, 32768, 128)):
-        q, k, v, do = (torch.randn((B, H, N, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-                       for _ in range(4))
+
+    def bf16(*shape):
+        return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    for (B, H, N, d, causal) in ((4, 16, 2048, 64, False), (1, 32, 8192, 128, False), (2, 16, 8192, 128, True)):
+        q, k, v, do = (bf16(B, H, N, d) for _ in range(4))
         o = torch.empty_like(q)
         lse = torch.empty((B, H, N), device=dev)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
         work = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
         sc = 1.0 / math.sqrt(d)
-        F = fwd_flops(B, H, N, d, True)
-        it = 10 if N <= 8192 else 4
-        tf = time_call(lambda: fa.fa_fwd(q, k, v, o, lse, sc, True, stream), iters=it)
-        tb = time_call(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, sc, True, work, stream), iters=it)
-        out[f"causal_b{B}_h{H}_n{N}_d{d}"] = {
-            "fwd_tflops": round(F / tf / 1e9, 1), "fwd_frac": round(F / tf / 1e9 / peaks["bf16_tflops"], 4),
-            "bwd_tflops": round(2.5 * F / tb / 1e9, 1),
-            "bwd_frac": round(2.5 * F / tb / 1e9 / peaks["bf16_tflops"], 4),
-            "fwd_bwd_tflops": round(3.5 * F / (tf + tb) / 1e9, 1)}
-        del q, k, v, do, o, dq, dk, dv, work
+        F = fwd_flops(B, H, N, d, causal)
+        it = 20 if N <= 2048 else 10
+        tf = time_call(lambda: fa.fa_fwd(q, k, v, o, lse, sc, causal, stream), iters=it)
+        tb, tk = time_call(lambda e: fa.fa_bwd_events(q, k, v, o, do, lse, dq, dk, dv, sc, causal, work, e, stream),
+                           iters=it, parts=True)
+        out[f"{'causal' if causal else 'noncausal'}_b{B}_h{H}_n{N}_d{d}"] = {
+            "fwd_tflops": round(F / tf / 1e9, 1), "fwd_frac": round(F / tf / 1e9 / pk, 4),
+            "bwd_tflops": round(2.5 * F / tb / 1e9, 1), "bwd_frac": round(2.5 * F / tb / 1e9 / pk, 4),
+            "bwd_kernel_tflops": round(2.5 * F / tk / 1e9, 1), "bwd_kernel_frac": round(2.5 * F / tk / 1e9 / pk, 4),
+            "fwd_bwd_tflops": round(3.5 * F / (tf + tb) / 1e9, 1),
+            "fwd_bwd_frac": round(3.5 * F / (tf + tb) / 1e9 / pk, 4),
+            "inputs": "N(0,1) from torch's seeded CUDA generator (timing only)"}
+        del q, k, v, do, o, dq, dk, dv, work, lse
     B, H, N, d = 2, 16, 16384, 128
     q8, k8, v8 = (torch.randn((B, H, N, d), generator=g, device=dev).mul_(100.0).clamp_(-448, 448)
                   .to(torch.float8_e4m3fn) for _ in range(3))
     o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, H, N), device=dev)
     F = fwd_flops(B, H, N, d, False)
-    try:
-        t8 = time_call(lambda: fa.fa_fwd_fp8(q8, k8, v8, 0.01, 0.01, 0.01, o, lse, 1.0 / math.sqrt(d), False, stream))
-        fp8_peak = 2.0 * peaks["bf16_tflops"]
-        out["fp8_fwd_b2_h16_n16384_d128"] = {
-            "tflops": round(F / t8 / 1e9, 1), "frac_of_fp8_peak": round(F / t8 / 1e9 / fp8_peak, 4),
-            "fp8_peak": fp8_peak, "fp8_peak_source": "2 x measured bf16 (nominal fp8:bf16 dense ratio)"}
-    except Exception as e:  # noqa: BLE001
-        out["fp8_fwd_b2_h16_n16384_d128"] = {"error": str(e)}
+    t8 = time_call(lambda: fa.fa_fwd_fp8(q8, k8, v8, 0.01, 0.01, 0.01, o, lse, 1.0 / math.sqrt(d), False, stream))
+    fp8_peak = 2.0 * pk
+    out["fp8_fwd_b2_h16_n16384_d128"] = {
+        "tflops": round(F / t8 / 1e9, 1), "frac_of_fp8_peak": round(F / t8 / 1e9 / fp8_peak, 4),
+        "fp8_peak": fp8_peak, "fp8_peak_source": "2 x measured bf16 (nominal fp8:bf16 dense ratio)"}
     del q8, k8, v8, o, lse
     # standard (materialising) attention against the fused forward on the same
     # inputs: the IO claim of the method, measured
     for (B, H, N, d) in ((4, 16, 2048, 64), (1, 32, 8192, 128)):
-        q, k, v = (torch.randn((B, H, N, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-                   for _ in range(3))
+        q, k, v = (bf16(B, H, N, d) for _ in range(3))
         o = torch.empty_like(q)
         lse = torch.empty((B, H, N), device=dev)
         work = torch.empty(fa.fa_fwd_standard_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
@@ -506,12 +569,11 @@ def extra_measurements(fa, torch, synth, dev, stream):
             "fused_hbm_bytes": B * H * (8 * N * d + 4 * N)}
         del q, k, v, o, lse, work
     # split-KV decode against a 16384-key cache: HBM-bound, K and V read once
-    # (2 GiB, well above L2, so back-to-back calls do not hit in cache)
+    # (2 GiB, well above L2; the flush write runs between calls as well)
     B, H, Nk, d = 8, 32, 16384, 128
-    k, v = (torch.randn((B, H, Nk, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-            for _ in range(2))
+    k, v = bf16(B, H, Nk, d), bf16(B, H, Nk, d)
     for Nq in (1, 4):
-        q = torch.randn((B, H, Nq, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        q = bf16(B, H, Nq, d)
         o = torch.empty_like(q)
         lse = torch.empty((B, H, Nq), device=dev)
         work = torch.empty(max(16, fa.fa_fwd_decode_workspace_size(B, H, Nq, Nk, d)), dtype=torch.uint8,
@@ -520,7 +582,9 @@ def extra_measurements(fa, torch, synth, dev, stream):
         nbytes = 2 * B * H * Nk * d * 2 + 2 * B * H * Nq * d * 2 + B * H * Nq * 4
         out[f"decode_b8_h32_nq{Nq}_nk16384_d128_causal"] = {
             "us": round(td * 1e3, 2), "gbs": round(nbytes / td / 1e6, 1),
-            "frac_of_hbm": round(nbytes / td / 1e6 / peaks["hbm_gbs"], 4), "bytes": nbytes}
+            "frac_of_measured_copy_bw": round(nbytes / td / 1e6 / peaks["hbm_gbs"], 4), "bytes": nbytes,
+            "note": "denominator: the measured STREAM-style copy bandwidth (read + write); a read-only "
+                    "stream can exceed it"}
     return out
 
 
@@ -535,57 +599,65 @@ def _oracle_threads():
 
 
 def oracle_sample(budget_s: float, seed: int = 4242):
-    """fwd+bwd of whole heads of the bench workload with the fp64 oracle until
-    the time budget is spent.  Returns (TFLOP/s, heads, seconds)."""
+    """fwd+bwd with the fp64 oracle on sample units of the bench workload until
+    the time budget is spent (at least one unit).  A unit is one head of the
+    workload's shape cut to its first n = min(N, CPU_SAMPLE_N) queries and
+    keys: under the causal mask those rows see exactly those keys, so the
+    unit's O, LSE and dQ rows are the workload's own, computed in the same
+    way.  Returns (TFLOP/s, units, seconds, n) with the unit's FLOPs counted
+    by the metric's formula."""
     import oracle
     import synth
 
-    B, H, N, d, causal = (WORKLOAD[k] for k in ("B", "H", "N", "d", "causal"))
-    inp = synth.attention_inputs(1, 4, N, d, seed=seed, want_f64=False)
+    d, causal = WORKLOAD["d"], WORKLOAD["causal"]
+    n = min(WORKLOAD["N"], CPU_SAMPLE_N)
+    inp = synth.attention_inputs(1, 4, n, d, seed=seed, want_f64=False)
     scale = 1.0 / math.sqrt(d)
-    heads, t0 = 0, time.perf_counter()
+    units, t0 = 0, time.perf_counter()
     while True:
-        h = heads % 4
-        qh, kh, vh, doh = (synth.head_f64(inp, n, 0, h) for n in ("q", "k", "v", "do"))
+        h = units % 4
+        qh, kh, vh, doh = (synth.head_f64(inp, nm, 0, h) for nm in ("q", "k", "v", "do"))
         oracle.head_backward(qh, kh, vh, doh, scale, causal)     # includes the forward
-        heads += 1
+        units += 1
         el = time.perf_counter() - t0
-        if el >= budget_s or heads >= B * H:
+        if el >= budget_s:
             break
-    flops = 3.5 * fwd_flops(1, 1, N, d, causal) * heads
-    return flops / el / 1e12, heads, el
+    flops = 3.5 * fwd_flops(1, 1, n, d, causal) * units
+    return flops / el / 1e12, units, el, n
 
 
 def cpu_baseline(args):
-    tflops, heads, el = oracle_sample(args.cpu_budget)
+    tflops, units, el, n = oracle_sample(args.cpu_budget)
     return {"value": tflops, "unit": "TFLOP/s", "cores": _oracle_threads(), "kind": "oracle",
-            "sample": f"{heads} of the 64 heads (fwd+bwd, fp64 numpy/OpenBLAS) of the bench workload in {el:.1f} s"}
+            "sample": f"{units} unit(s) of one head cut to its first {n} queries and keys "
+                      f"(fwd+bwd, fp64 numpy/OpenBLAS, {'causal' if WORKLOAD['causal'] else 'non-causal'}, "
+                      f"d={WORKLOAD['d']}) in {el:.1f} s; FLOPs by the metric's formula for the unit"}
 
 
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return
-    per_step, heads_total, t_total = [], 0, 0.0
+    per_step, units_total, t_total, n = [], 0, 0.0, 0
     for _ in range(args.warmup):
         oracle_sample(0.0)
     for _ in range(args.steps):
-        tf, heads, el = oracle_sample(args.ref_step_budget)
+        _, units, el, n = oracle_sample(args.ref_step_budget)
         per_step.append(el)
-        heads_total += heads
+        units_total += units
         t_total += el
-    F = 3.5 * fwd_flops(1, 1, WORKLOAD["N"], WORKLOAD["d"], WORKLOAD["causal"]) * heads_total
+    F = 3.5 * fwd_flops(1, 1, n, WORKLOAD["d"], WORKLOAD["causal"]) * units_total
     value = F / t_total / 1e12
     cores = _oracle_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / max(1, args.steps),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) Philox, rounded to bf16, evaluated in fp64)",
         "config": {"workload": WORKLOAD_NAME, **WORKLOAD},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: whole heads (fwd+bwd) for {args.ref_step_budget:.1f} s; "
-                                   f"{heads_total} heads in total"},
+                         "sample": f"each step: units of one head cut to its first {n} queries and keys "
+                                   f"(fwd+bwd) for {args.ref_step_budget:.1f} s; {units_total} units in total"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -603,12 +675,15 @@ def main():
     ap.add_argument("--ref-step-budget", type=float, default=1.0)
     ap.add_argument("--shape", default="", help="B,H,N,d of another workload (default: the bench workload)")
     ap.add_argument("--causal", action="store_true")
-    ap.add_argument("--case", choices=["decode", "standard"], default="",
+    ap.add_argument("--noncausal", action="store_true")
+    ap.add_argument("--case", choices=["decode", "standard", "fp8"], default="",
                     help="profile one path on --shape instead of the bench step")
     ap.add_argument("--nq", type=int, default=1, help="queries per head for --case decode")
     ap.add_argument("--clock-window", type=float, default=1.5,
                     help="seconds of steps run under the clock sampler before the timed region")
     args = ap.parse_args()
+    if args.causal and args.noncausal:
+        ap.error("--causal and --noncausal exclude each other")
     if args.case:
         if not args.shape:
             ap.error("--case needs --shape")
@@ -617,6 +692,10 @@ def main():
     apply_shape(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args))
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -96,6 +96,9 @@ def fa_bwd_events(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, w
     _check_tensors((B, H, N), torch.float32, lse)
     if len(events) != 4:
         raise ValueError("fa_bwd_events takes four events")
+    for e in events:
+        if int(e.cuda_event) == 0:         # torch creates the CUDA event at its first record
+            e.record(torch.cuda.current_stream() if stream is None else stream)
     arr = (ctypes.c_void_p * 4)(*(int(e.cuda_event) for e in events))
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     check(lib.fa_bwd_events(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),

@@ -154,3 +154,27 @@ def test_bwd_scale_zero(d, causal):
     assert np.all(ref[0] == 0.0) and np.all(ref[1] == 0.0)
     e = gu.rel_fro(dv, ref[2])
     assert e <= gu.GRAD_REL_FRO, e
+
+
+@pytest.mark.parametrize("d,causal", [(64, False), (128, True)])
+def test_bwd_events_matches_fa_bwd_and_orders_its_events(d, causal):
+    """fa_bwd_events computes what fa_bwd computes (dK, dV byte for byte; dQ
+    within the tolerance, its fp32 atomics reorder) and its four events bound
+    the preprocess, the main kernel and the dQ conversion in that order."""
+    B, H, N = 2, 3, 1000
+    inp = synth.attention_inputs(B, H, N, d, seed=1249 + d, want_f64=False)
+    q, k, v, do = _device_inputs(inp)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = fa.attention_forward(q, k, v, scale=scale, causal=causal)
+    ref = fa.attention_backward(q, k, v, o, do, lse, scale=scale, causal=causal)
+    outs = [torch.empty_like(q) for _ in range(3)]
+    work = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    fa.fa_bwd_events(q, k, v, o, do, lse, *outs, scale, causal, work, ev)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[1].view(torch.int16), ref[1].view(torch.int16))
+    assert torch.equal(outs[2].view(torch.int16), ref[2].view(torch.int16))
+    assert gu.rel_fro(gu.to_f64(outs[0]), gu.to_f64(ref[0])) <= 1e-3
+    parts = [ev[i].elapsed_time(ev[i + 1]) for i in range(3)]
+    assert all(p >= 0.0 for p in parts) and parts[1] > 0.0
+    assert fa.fa_device_status() == (0, 0)
