@@ -18,6 +18,12 @@ import random
 import pytest
 
 
+import kernel_constants as kc
+
+K = kc.barrier_counts("fa_bwd_dq.cu")
+WARPS_PER_GROUP = 4      # a model agent for an elementwise group stands for its 4 warps
+
+
 class Bar:
     def __init__(self, name, count):
         self.name, self.count, self.arrivals, self.completed = name, count, 0, 0
@@ -41,13 +47,15 @@ class Model:
     def __init__(self, T, nst, rng, plant=None):
         self.T, self.nst, self.rng, self.plant = T, nst, rng, plant
         B = Bar
-        self.qdo_full = B("qdo_full", 1)
-        self.k_full = [B(f"k_full{s}", 1) for s in range(nst)]
-        self.v_full = [B(f"v_full{s}", 1) for s in range(nst)]
-        self.kv_empty = [B(f"kv_empty{s}", 1) for s in range(nst)]
-        self.s_full, self.dp_full = B("s_full", 1), B("dp_full", 1)
-        self.s_free, self.dp_free = B("s_free", 1), B("dp_free", 1)
-        self.ds_full, self.ds_free, self.final_ = B("ds_full", 1), B("ds_free", 1), B("final", 1)
+        g = lambda n: kc.per_agent(K[n], 2 * WARPS_PER_GROUP, n)  # noqa: E731  (one agent: both groups)
+        self.qdo_full = B("qdo_full", K["qdo_full"])
+        self.k_full = [B(f"k_full{s}", K["k_full"]) for s in range(nst)]
+        self.v_full = [B(f"v_full{s}", K["v_full"]) for s in range(nst)]
+        self.kv_empty = [B(f"kv_empty{s}", K["kv_empty"]) for s in range(nst)]
+        self.s_full, self.dp_full = B("s_full", K["s_full"]), B("dp_full", K["dp_full"])
+        self.s_free, self.dp_free = B("s_free", g("s_free")), B("dp_free", g("dp_free"))
+        self.ds_full, self.ds_free = B("ds_full", g("ds_full")), B("ds_free", K["ds_free"])
+        self.final_ = B("final", K["final_"])
         self.speeds = {}
         self.pipe, self.tma = [], []
         self.exec = {"S": 0, "dP": 0, "dQ": 0}
@@ -162,7 +170,8 @@ class Model:
         raise Violation("step limit")
 
 
-@pytest.mark.parametrize("nst", [2, 4])          # ring depth at d = 128 and d = 64
+@pytest.mark.parametrize("nst", [kc.ring_depth("fa_bwd_dq.cu", "kNST", 128),
+                                 kc.ring_depth("fa_bwd_dq.cu", "kNST", 64)])   # ring depth at d = 128, 64
 @pytest.mark.parametrize("T", [1, 2, 3, 5, 16])
 def test_protocol_holds_under_random_interleavings(T, nst):
     for seed in range(60):
@@ -178,3 +187,11 @@ def test_protocol_model_catches_a_planted_missing_wait():
         except Violation:
             caught += 1
     assert caught > 0
+
+
+def test_model_counts_are_the_kernels():
+    """One arrive per warp of both elementwise groups on s_free, dp_free and
+    ds_full (the model's single elementwise agent), one per commit elsewhere."""
+    assert K["s_free"] == K["dp_free"] == K["ds_full"] == 2 * WARPS_PER_GROUP
+    assert all(K[n] == 1 for n in ("qdo_full", "k_full", "v_full", "kv_empty", "s_full", "dp_full", "ds_free",
+                                   "final_"))

@@ -28,7 +28,13 @@ import random
 
 import pytest
 
-NST = 2  # Q / dO / statistics ring depth of the backward
+import kernel_constants as kc
+
+NST = kc.ring_depth("fa_bwd.cu", "kNST")   # Q / dO / statistics ring depth of the backward
+# Arrive counts of the kernel's barriers.  A model agent for a P/dS group or
+# the dQ group stands for that group's 4 warps, each of which arrives once.
+K = kc.barrier_counts("fa_bwd.cu")
+WARPS_PER_GROUP = 4
 
 
 class Bar:
@@ -54,16 +60,20 @@ class Model:
     def __init__(self, n_iter, rng, plant=None, d=64):
         self.n, self.rng, self.plant, self.d = n_iter, rng, plant, d
         B = Bar
-        self.kv_full = B("kv_full", 1)
-        self.kv_tmem = B("kv_tmem", 2)
-        self.qdo_full = [B(f"qdo_full{s}", 1) for s in range(NST)]
-        self.qdo_empty = [B(f"qdo_empty{s}", 3) for s in range(NST)]   # MMA commit + 2 groups
-        self.s_ready, self.dp_ready = B("s_ready", 1), B("dp_ready", 1)
-        self.p_ready, self.ds_ready = B("p_ready", 2), B("ds_ready", 2)
-        self.ds_free, self.dq_ready, self.dq_free = B("ds_free", 1), B("dq_ready", 1), B("dq_free", 1)
-        self.dq_staged = [B("dq_staged0", 1), B("dq_staged1", 1)]
-        self.dq_stage_free = [B("dq_stage_free0", 1), B("dq_stage_free1", 1)]
-        self.final_ = B("final", 1)
+        g = lambda n: kc.per_agent(K[n], WARPS_PER_GROUP, n)  # noqa: E731
+        self.kv_full = B("kv_full", K["kv_full"])
+        self.kv_tmem = B("kv_tmem", g("kv_tmem"))
+        self.qdo_full = [B(f"qdo_full{s}", K["qdo_full"]) for s in range(NST)]
+        # MMA commit + the P/dS groups
+        self.qdo_empty = [B(f"qdo_empty{s}", 1 + kc.per_agent(K["qdo_empty"] - 1, WARPS_PER_GROUP, "qdo_empty"))
+                          for s in range(NST)]
+        self.s_ready, self.dp_ready = B("s_ready", K["s_ready"]), B("dp_ready", K["dp_ready"])
+        self.p_ready, self.ds_ready = B("p_ready", g("p_ready")), B("ds_ready", g("ds_ready"))
+        self.ds_free, self.dq_ready = B("ds_free", K["ds_free"]), B("dq_ready", K["dq_ready"])
+        self.dq_free = B("dq_free", g("dq_free"))
+        self.dq_staged = [B(f"dq_staged{b}", g("dq_staged")) for b in range(2)]
+        self.dq_stage_free = [B(f"dq_stage_free{b}", K["dq_stage_free"]) for b in range(2)]
+        self.final_ = B("final", K["final_"])
         self.speeds = {}
         self.pipe, self.tma, self.reduce_reads = [], [], []
         self.exec = {k: 0 for k in ("S", "dP", "dV", "dK", "dQ")}   # products executed
@@ -271,3 +281,14 @@ def test_protocol_model_catches_a_planted_missing_wait(d):
         except Violation:
             caught += 1
     assert caught > 0
+
+
+def test_model_counts_are_the_kernels():
+    """The kernel's counts map onto the model's agents: one arrive per warp of
+    the two P/dS groups (and of the dQ group), one for each commit."""
+    assert K["p_ready"] == K["ds_ready"] == K["kv_tmem"] == 2 * WARPS_PER_GROUP
+    assert K["qdo_empty"] == 1 + 2 * WARPS_PER_GROUP
+    assert K["dq_free"] == K["dq_staged"] == WARPS_PER_GROUP
+    assert all(K[n] == 1 for n in ("kv_full", "qdo_full", "s_ready", "dp_ready", "ds_free", "dq_ready",
+                                   "final_", "dq_stage_free"))
+    assert NST >= 2

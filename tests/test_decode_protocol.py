@@ -18,7 +18,11 @@ import random
 
 import pytest
 
-NS = 3  # K/V ring depth of the decode kernel
+import kernel_constants as kc
+
+NS = kc.ring_depth("fa_decode.cu", "kNS")   # K/V ring depth of the decode kernel
+K = kc.barrier_counts("fa_decode.cu")
+WARPS_PER_ROLE = 4      # a model agent for the softmax or epilogue role stands for its 4 warps
 
 
 class Bar:
@@ -44,17 +48,15 @@ class Model:
     def __init__(self, nts, rescale, rng, plant=None):
         self.nts, self.rescale, self.rng, self.plant = nts, rescale, rng, plant
         B = Bar
-        self.q_full = [B("q_full0", 1), B("q_full1", 1)]
-        self.q_empty = [B("q_empty0", 1), B("q_empty1", 1)]
-        self.kv_full = [B(f"kv_full{s}", 1) for s in range(NS)]
-        self.kv_empty = [B(f"kv_empty{s}", 1) for s in range(NS)]
-        self.s_full = [B("s_full0", 1), B("s_full1", 1)]
-        self.s_free = [B("s_free0", 1), B("s_free1", 1)]
-        self.p_full = [B("p_full0", 1), B("p_full1", 1)]
-        self.pv_done = [B("pv_done0", 1), B("pv_done1", 1)]
-        self.o_full = [B("o_full0", 1), B("o_full1", 1)]
-        self.o_free = [B("o_free0", 1), B("o_free1", 1)]
-        self.stats_full = [B("stats_full0", 1), B("stats_full1", 1)]
+        g = lambda n: kc.per_agent(K[n], WARPS_PER_ROLE, n)  # noqa: E731
+        two = lambda n, c: [B(f"{n}{i}", c) for i in range(2)]  # noqa: E731
+        self.q_full, self.q_empty = two("q_full", K["q_full"]), two("q_empty", K["q_empty"])
+        self.kv_full = [B(f"kv_full{s}", K["kv_full"]) for s in range(NS)]
+        self.kv_empty = [B(f"kv_empty{s}", K["kv_empty"]) for s in range(NS)]
+        self.s_full, self.s_free = two("s_full", K["s_full"]), two("s_free", g("s_free"))
+        self.p_full, self.pv_done = two("p_full", g("p_full")), two("pv_done", K["pv_done"])
+        self.o_full, self.o_free = two("o_full", K["o_full"]), two("o_free", g("o_free"))
+        self.stats_full = two("stats_full", g("stats_full"))
         self.speeds = {}
         self.pipe, self.tma = [], []
         self.s_exec = 0            # S^T products executed (ring index order)
@@ -235,3 +237,10 @@ def test_protocol_model_catches_a_planted_missing_wait():
         except Violation:
             caught += 1
     assert caught > 0
+
+
+def test_model_counts_are_the_kernels():
+    """One arrive per warp of the softmax role (s_free, p_full, red) and of the
+    epilogue role (o_free, stats_full), one per commit or TMA elsewhere."""
+    assert K["s_free"] == K["p_full"] == K["red"] == K["o_free"] == K["stats_full"] == WARPS_PER_ROLE
+    assert all(K[n] == 1 for n in ("q_full", "q_empty", "kv_full", "kv_empty", "s_full", "pv_done", "o_full"))

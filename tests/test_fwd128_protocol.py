@@ -18,7 +18,11 @@ import random
 
 import pytest
 
-NST = 2  # K/V ring depth at d = 128 (32 KB tiles)
+import kernel_constants as kc
+
+NST = kc.ring_depth("fa_fwd.cu", "kNST", 128)   # K/V ring depth at d = 128 (32 KB tiles)
+K = kc.barrier_counts("fa_fwd.cu")
+WARPS_PER_GROUP = 4      # a model agent for a softmax group stands for its 4 warps
 
 
 class Bar:
@@ -44,13 +48,13 @@ class Model:
     def __init__(self, T, rescale, rng, plant=None):
         self.T, self.rescale, self.rng, self.plant = T, rescale, rng, plant
         B = Bar
-        self.q = B("q", 1)
-        self.k_full = [B(f"k_full{s}", 1) for s in range(NST)]
-        self.v_full = [B(f"v_full{s}", 1) for s in range(NST)]
-        self.kv_empty = [B(f"kv_empty{s}", 1) for s in range(NST)]
-        self.s_full = [B("s_full0", 1), B("s_full1", 1)]
-        self.p_full = [B("p_full0", 1), B("p_full1", 1)]
-        self.o_final = [B("o_final0", 1), B("o_final1", 1)]
+        self.q = B("q", K["q"])
+        self.k_full = [B(f"k_full{s}", K["k_full"]) for s in range(NST)]
+        self.v_full = [B(f"v_full{s}", K["v_full"]) for s in range(NST)]
+        self.kv_empty = [B(f"kv_empty{s}", K["kv_empty"]) for s in range(NST)]
+        self.s_full = [B(f"s_full{g}", K["s_full"]) for g in range(2)]
+        self.p_full = [B(f"p_full{g}", kc.per_agent(K["p_full"], WARPS_PER_GROUP, "p_full")) for g in range(2)]
+        self.o_final = [B(f"o_final{g}", K["o_final"]) for g in range(2)]
         self.speeds = {}
         self.pipe, self.tma = [], []
         self.s_exec = [0, 0]        # S_g tiles executed
@@ -199,3 +203,9 @@ def test_protocol_model_catches_a_planted_missing_wait():
         except Violation:
             caught += 1
     assert caught > 0
+
+
+def test_model_counts_are_the_kernels():
+    assert K["p_full"] == WARPS_PER_GROUP
+    assert all(K[n] == 1 for n in ("q", "k_full", "v_full", "kv_empty", "s_full", "o_final"))
+    assert NST == kc.ring_depth("fa_fwd.cu", "kNST", 128)

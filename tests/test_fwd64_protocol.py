@@ -28,7 +28,11 @@ import random
 
 import pytest
 
-NST = 4  # K/V ring depth of the d = 64 kernel
+import kernel_constants as kc
+
+NST = kc.ring_depth("fa_fwd64.cu", "kD64NST")   # K/V ring depth of the d = 64 kernel
+K = kc.barrier_counts("fa_fwd64.cu")
+WARPS_PER_GROUP = 4      # a model agent for a softmax group stands for its 4 warps
 
 
 class Bar:
@@ -55,16 +59,15 @@ class Model:
     def __init__(self, items, rng, planted_bug=False):
         self.items, self.rng, self.bug = items, rng, planted_bug
         B = Bar
-        self.q_full = [B("q_full0", 1), B("q_full1", 1)]
-        self.q_empty = [B("q_empty0", 2), B("q_empty1", 2)]
-        self.k_full = [B(f"k_full{s}", 1) for s in range(NST)]
-        self.v_full = [B(f"v_full{s}", 1) for s in range(NST)]
-        self.kv_empty = [B(f"kv_empty{s}", 2) for s in range(NST)]
-        self.s_full = [B("s_full0", 1), B("s_full1", 1)]
-        self.s_free = [B("s_free0", 1), B("s_free1", 1)]
-        self.p_full = [B("p_full0", 1), B("p_full1", 1)]
-        self.pv_done = [B("pv_done0", 1), B("pv_done1", 1)]
-        self.o_final = [B("o_final0", 1), B("o_final1", 1)]
+        g = lambda n: kc.per_agent(K[n], WARPS_PER_GROUP, n)  # noqa: E731
+        two = lambda n, c: [B(f"{n}{i}", c) for i in range(2)]  # noqa: E731
+        self.q_full, self.q_empty = two("q_full", K["q_full"]), two("q_empty", K["q_empty"])  # both MMA warps
+        self.k_full = [B(f"k_full{s}", K["k_full"]) for s in range(NST)]
+        self.v_full = [B(f"v_full{s}", K["v_full"]) for s in range(NST)]
+        self.kv_empty = [B(f"kv_empty{s}", K["kv_empty"]) for s in range(NST)]   # both MMA warps
+        self.s_full, self.s_free = two("s_full", K["s_full"]), two("s_free", g("s_free"))
+        self.p_full, self.pv_done = two("p_full", g("p_full")), two("pv_done", K["pv_done"])
+        self.o_final = two("o_final", K["o_final"])
         self.speeds = {}
         self.pipe = []          # in-order tensor pipe: ("mma", info) | ("commit", bar)
         self.tma = []           # outstanding loads: bars to arrive on
@@ -299,3 +302,11 @@ def test_kernel_items_cover_every_q_tile_once():
             its = kernel_items(BH, N, causal, sms, cta)
             tiles += sum((T0 > 0) + (T1 > 0) for T0, T1 in its)
         assert tiles == BH * n_qt, (BH, N, causal, sms, tiles)
+
+
+def test_model_counts_are_the_kernels():
+    """Each K/V stage and Q buffer is released by both MMA-issuing warps (one
+    per Q-tile slot); S is freed and P published by the 4 warps of a group."""
+    assert K["kv_empty"] == K["q_empty"] == 2
+    assert K["s_free"] == K["p_full"] == WARPS_PER_GROUP
+    assert all(K[n] == 1 for n in ("q_full", "k_full", "v_full", "s_full", "pv_done", "o_final"))
