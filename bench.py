@@ -549,7 +549,17 @@ def extra_measurements(fa, torch, dev, stream, flush):
     out["fp8_fwd_b2_h16_n16384_d128"] = {
         "tflops": round(F / t8 / 1e9, 1), "frac_of_fp8_peak": round(F / t8 / 1e9 / fp8_peak, 4),
         "fp8_peak": fp8_peak, "fp8_peak_source": "2 x measured bf16 (nominal fp8:bf16 dense ratio)"}
-    del q8, k8, v8, o, lse
+    # its backward: e4m3 Q, K, V widened exactly to bf16, the bf16 backward kernels
+    do = bf16(B, H, N, d)
+    dq, dk, dv = (torch.empty_like(do) for _ in range(3))
+    work = torch.empty(fa.fa_bwd_fp8_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    tb8 = time_call(lambda: fa.fa_bwd_fp8(q8, k8, v8, 0.01, 0.01, 0.01, o, do, lse, dq, dk, dv, 1.0 / math.sqrt(d),
+                                          False, work, stream))
+    out["fp8_bwd_b2_h16_n16384_d128"] = {
+        "tflops": round(2.5 * F / tb8 / 1e9, 1), "frac_of_bf16_peak": round(2.5 * F / tb8 / 1e9 / pk, 4),
+        "fwd_bwd_tflops": round(3.5 * F / (t8 + tb8) / 1e9, 1),
+        "note": "the five products run on bf16 tensor cores (exact widening of the e4m3 inputs)"}
+    del q8, k8, v8, o, lse, do, dq, dk, dv, work
     # standard (materialising) attention against the fused forward on the same
     # inputs: the IO claim of the method, measured
     for (B, H, N, d) in ((4, 16, 2048, 64), (1, 32, 8192, 128)):

@@ -16,7 +16,7 @@ from ._lib import FA_OK, FAError, LIB_PATH, STATUS_CODES, STATUS_NAMES, check, l
 
 __all__ = [
     "FAError", "LIB_PATH", "fa_fwd", "fa_fwd_fp8", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size",
-    "fa_bwd_events", "fa_fwd_plan", "fa_get_device_status", "fa_device_status", "fa_fwd_decode", "fa_fwd_decode_workspace_size", "attention_decode",
+    "fa_bwd_events", "fa_fwd_plan", "fa_bwd_fp8", "fa_bwd_fp8_workspace_size", "attention_backward_fp8", "fa_get_device_status", "fa_device_status", "fa_fwd_decode", "fa_fwd_decode_workspace_size", "attention_decode",
     "fa_fwd_standard", "fa_fwd_standard_workspace_size", "attention_forward_standard",
     "fa_watchdog_selftest", "attention_forward", "attention_backward", "attention_forward_fp8", "lib",
     "STATUS_NAMES", "STATUS_CODES", "strerror",
@@ -104,6 +104,33 @@ def fa_bwd_events(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, w
     check(lib.fa_bwd_events(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
                             B, H, N, d, float(scale), int(bool(causal)), _ptr(workspace), wbytes, arr,
                             _stream_ptr(stream)))
+
+
+def fa_bwd_fp8_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    n = int(lib.fa_bwd_fp8_workspace_size(B, H, N, d))
+    if n == ctypes.c_size_t(-1).value:
+        raise FAError(1, "invalid shape for fa_bwd_fp8_workspace_size (d must be 128)")
+    return n
+
+
+def _check_e4m3(shape, *ts):
+    for t in ts:
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or tuple(t.shape) != shape \
+                or not t.is_contiguous() or t.device.type != "cuda":
+            raise ValueError("e4m3 inputs must be contiguous CUDA uint8/float8_e4m3fn [B,H,N,d]")
+
+
+def fa_bwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, o, do, lse, dq, dk, dv, scale: float, causal: bool,
+               workspace, stream=None) -> None:
+    """dQ, dK, dV (real units) <- backward of the e4m3 forward; workspace is a CUDA uint8 tensor."""
+    B, H, N, d = _shape(q8)
+    _check_e4m3((B, H, N, d), q8, k8, v8)
+    _check_tensors((B, H, N, d), torch.bfloat16, o, do, dq, dk, dv)
+    _check_tensors((B, H, N), torch.float32, lse)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(lib.fa_bwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_descale), float(k_descale), float(v_descale),
+                         _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, float(scale),
+                         int(bool(causal)), _ptr(workspace), wbytes, _stream_ptr(stream)))
 
 
 def fa_fwd_plan(B: int, H: int, N: int, d: int, causal: bool):
@@ -230,4 +257,16 @@ def attention_backward(q, k, v, o, do, lse, scale: float | None = None, causal: 
         workspace = torch.empty(max(1, fa_bwd_workspace_size(B, H, N, d)), dtype=torch.uint8, device=q.device)
     fn = fa_bwd_deterministic if deterministic else fa_bwd
     fn(q, k, v, o, do, lse, dq, dk, dv, _default_scale(d) if scale is None else scale, causal, workspace, stream)
+    return dq, dk, dv
+
+
+def attention_backward_fp8(q8, k8, v8, q_descale, k_descale, v_descale, o, do, lse, scale: float | None = None,
+                           causal: bool = False, workspace=None, stream=None):
+    """(dQ, dK, dV) bf16 of the e4m3 forward, allocating outputs and workspace with torch."""
+    B, H, N, d = _shape(q8)
+    dq, dk, dv = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device) for _ in range(3))
+    if workspace is None:
+        workspace = torch.empty(max(256, fa_bwd_fp8_workspace_size(B, H, N, d)), dtype=torch.uint8, device=q8.device)
+    fa_bwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, o, do, lse, dq, dk, dv,
+               _default_scale(d) if scale is None else scale, causal, workspace, stream)
     return dq, dk, dv

@@ -58,6 +58,10 @@ def _load() -> ctypes.CDLL:
     lib.fa_fwd_standard.restype = i
     lib.fa_fwd_standard_workspace_size.argtypes = [i, i, i, i]
     lib.fa_fwd_standard_workspace_size.restype = sz
+    lib.fa_bwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_bwd_fp8.restype = i
+    lib.fa_bwd_fp8_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_bwd_fp8_workspace_size.restype = sz
     lib.fa_bwd_events.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz,
                                   ctypes.POINTER(vp), vp]
     lib.fa_bwd_events.restype = i

@@ -338,10 +338,33 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
 }
 
 namespace {
+// e4m3 inputs of the backward of fa_fwd_fp8 (NULL: bf16 inputs)
+struct Fp8Inputs {
+  const void* q8;
+  const void* k8;
+  const void* v8;
+  float qd, kd, vd;
+};
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                      void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                      void* workspace, size_t workspace_bytes, void* stream, bool deterministic,
-                     void* const* events);
+                     void* const* events, const Fp8Inputs* fp8 = nullptr);
+
+// Workspace of the e4m3 backward: the bf16 backward's, then the bf16 widening
+// of Q, K and V (each 256-byte aligned).
+struct Fp8WsLayout {
+  size_t q_off, k_off, v_off, total;
+};
+Fp8WsLayout fp8_ws_layout(long long BH, int N, int d) {
+  Fp8WsLayout w{};
+  const size_t t = static_cast<size_t>(BH) * N * d * 2;
+  const size_t a = (t + 255) / 256 * 256;
+  w.q_off = (ws_layout(BH, N, d).total + 255) / 256 * 256;
+  w.k_off = w.q_off + a;
+  w.v_off = w.k_off + a;
+  w.total = w.v_off + t;
+  return w;
+}
 }  // namespace
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
@@ -359,6 +382,22 @@ fa_status fa_bwd_events(const void* q, const void* k, const void* v, const void*
                     false, events);
 }
 
+size_t fa_bwd_fp8_workspace_size(int B, int H, int N, int d) {
+  bool empty = false;
+  if (check_shape(B, H, N, d, 1.0f, 0, &empty) != FA_OK || d != 128) return static_cast<size_t>(-1);
+  if (empty) return 0;
+  return fp8_ws_layout(static_cast<long long>(B) * H, N, d).total;
+}
+
+fa_status fa_bwd_fp8(const void* q8, const void* k8, const void* v8, float q_descale, float k_descale,
+                     float v_descale, const void* o, const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                     int B, int H, int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  const Fp8Inputs in{q8, k8, v8, q_descale, k_descale, v_descale};
+  return bwd_common(q8, k8, v8, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes,
+                    stream, false, nullptr, &in);
+}
+
 fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,
                                const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                                float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
@@ -372,21 +411,43 @@ namespace {
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                      void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                      void* workspace, size_t workspace_bytes, void* stream, bool deterministic,
-                     void* const* events) {
+                     void* const* events, const Fp8Inputs* fp8) {
   bool empty = false;
   fa_status st = check_shape(B, H, N, d, scale, causal, &empty);
   if (st != FA_OK) return st;
+  if (fp8 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (fp8 && !(std::isfinite(fp8->qd) && std::isfinite(fp8->kd) && std::isfinite(fp8->vd) && fp8->qd > 0 &&
+               fp8->kd > 0 && fp8->vd > 0))
+    return FA_ERR_INVALID_ARG;
   if (empty) return FA_OK;
   if (causal && !grid_fits(static_cast<long long>(B) * H, N)) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   const int BH = B * H;
   const WsLayout wl = ws_layout(BH, N, d);
-  if (!workspace || workspace_bytes < wl.total) return FA_ERR_WORKSPACE;
+  const size_t need = fp8 ? fp8_ws_layout(BH, N, d).total : wl.total;
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
       !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(workspace, 16) || !aligned(lse, 4))
     return FA_ERR_ALIGNMENT;
   uint32_t* status = nullptr;
   if ((st = current_device(&status)) != FA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (fp8) {
+    // The bf16 kernels run on the exact bf16 values of the e4m3 bytes; the
+    // descales are folded into the score, dP, dK and dQ factors below.
+    const Fp8WsLayout fl = fp8_ws_layout(BH, N, d);
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    const long long n16 = static_cast<long long>(BH) * N * d / 16;
+    void* wq = wsb + fl.q_off;
+    void* wk = wsb + fl.k_off;
+    void* wv = wsb + fl.v_off;
+    if (fa::launch_widen_e4m3(q, wq, n16, cs) != cudaSuccess || fa::launch_widen_e4m3(k, wk, n16, cs) != cudaSuccess ||
+        fa::launch_widen_e4m3(v, wv, n16, cs) != cudaSuccess)
+      return FA_ERR_LAUNCH;
+    q = wq;
+    k = wk;
+    v = wv;
+  }
   CUtensorMap tq, tk, tv, tdo;
   if (!make_map(&tq, q, false, d, N, BH) || !make_map(&tk, k, false, d, N, BH) ||
       !make_map(&tv, v, false, d, N, BH) || !make_map(&tdo, dO, false, d, N, BH))
@@ -406,14 +467,15 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   a.N = N;
   a.Np = static_cast<int>(padded_rows(N));
   a.BH = BH;
-  a.c_log2 = scale * kLog2e;
-  a.scale = scale;
+  a.c_log2 = scale * kLog2e * (fp8 ? fp8->qd * fp8->kd : 1.0f);
+  a.dp_scale = fp8 ? fp8->vd : 1.0f;
+  a.dk_scale = scale * (fp8 ? fp8->qd : 1.0f);
+  a.dq_scale = scale * (fp8 ? fp8->kd : 1.0f);
   a.head_group = head_group(8ll * N * d, BH);   // Q, dO (bf16) and the fp32 dQ rows of a head
   CUtensorMap tdq;
   if (!make_map_dq(&tdq, a.dq_acc, d, N, BH)) return FA_ERR_LAUNCH;
   return launch_status(
-      fa::launch_bwd(tq, tk, tv, tdo, tdq, a, d, causal != 0, deterministic, events,
-                     static_cast<cudaStream_t>(stream)));
+      fa::launch_bwd(tq, tk, tv, tdo, tdq, a, d, causal != 0, deterministic, events, cs));
 }
 }  // namespace
 

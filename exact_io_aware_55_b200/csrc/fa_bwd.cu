@@ -42,6 +42,7 @@
 // the untransposed dQ tile has its own columns [384, 448), and copies of K_j
 // and V_j (the A operands of S^T and dP^T) sit in [448, 480) and [480, 512).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -115,6 +116,34 @@ __global__ void __launch_bounds__(256) bwd_dq_final_kernel(const float* __restri
     o.z = pack_bf16x2(y.x * scale, y.y * scale);
     o.w = pack_bf16x2(y.z * scale, y.w * scale);
     reinterpret_cast<uint4*>(dq)[t] = o;
+  }
+}
+
+// ------------------------------------------------------- e4m3 -> bf16
+// Every e4m3 value (normal or subnormal, |x| <= 448) is exactly an f16 value
+// and, with at most 4 significant bits, exactly a bf16 value: e4m3 -> f16x2
+// (hardware cvt) -> f32 -> bf16x2 loses nothing.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t x) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(x));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16x2(f.x, f.y);
+}
+
+__global__ void __launch_bounds__(256) widen_e4m3_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                         long long n16) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n16; t += stride) {
+    const uint4 x = src[t];
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      o[2 * k] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w[k] & 0xffffu));
+      o[2 * k + 1] = e4m3x2_to_bf16x2(static_cast<uint16_t>(w[k] >> 16));
+    }
+    dst[2 * t] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * t + 1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 
@@ -478,7 +507,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (it > 0 && !mbar_wait_warp(&bars->ds_free, (it - 1) & 1, wc, WAIT_BWD_DS_FREE)) { ok = false; break; }
       tc_fence_after();
       // 64 queries = 128 bytes = one full row of chunk h, eight 16-byte units;
-      // dP^T in two 32-column pieces.
+      // dP^T in two 32-column pieces.  dP - D = dp_scale * dP^T(as computed) - D.
+      const float2 dps = make_float2(args.dp_scale, args.dp_scale);
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         uint32_t r[32];
@@ -489,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t = 16 * q + t2;
           const float4 nd4 = *reinterpret_cast<const float4*>(snd + 4 * (t >> 1));
           const float2 nd = (t & 1) ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
-          const float2 dpm = fadd2(make_float2(__uint_as_float(r[2 * t2]), __uint_as_float(r[2 * t2 + 1])), nd);
+          const float2 dpm = ffma2(make_float2(__uint_as_float(r[2 * t2]), __uint_as_float(r[2 * t2 + 1])), dps, nd);
           const float2 ds = fmul2(pf[t], dpm);
           w[t2] = pack_bf16x2(ds.x, ds.y);
         }
@@ -515,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(h == 0 ? args.dv : args.dk) + (size_t(bh) * N + kv) * D;
       const uint32_t src = lane_base + (h == 0 ? S::kColDV : S::kColDK);
-      const float f = (h == 0) ? 1.0f : args.scale;   // dK = scale * dS^T Q
+      const float f = (h == 0) ? 1.0f : args.dk_scale;   // dK = scale * dS^T Q
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         uint32_t r[32];
@@ -663,7 +693,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     const long long n8 = (long long)a.BH * a.N * D / 8;
     const int fin_blocks = int(std::min<long long>((n8 + 255) / 256, 148LL * 8));
     bwd_dq_final_kernel<<<fin_blocks, 256, 0, stream>>>(a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq), n8,
-                                                        a.scale);
+                                                        a.dq_scale);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = mark(3);
@@ -671,6 +701,13 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 }
 
 }  // namespace
+
+cudaError_t launch_widen_e4m3(const void* src, void* dst, long long n16, cudaStream_t stream) {
+  if (n16 <= 0) return cudaSuccess;
+  const int blocks = int(std::min<long long>((n16 + 255) / 256, 148LL * 8));
+  widen_e4m3_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                        const CUtensorMap& tdq, const BwdArgs& a, int d, bool causal, bool deterministic,

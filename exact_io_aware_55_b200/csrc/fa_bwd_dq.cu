@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t srow = size_t(bh) * args.Np + size_t(q);
     const float nl = args.neg_lse2[srow];             // -LSE*log2e (-inf on padded rows)
     const float nd = args.neg_dvec[srow];             // -D
-    const float cl = args.c_log2, scale = args.scale;
+    const float cl = args.c_log2, scale = args.dq_scale;
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const bool diag = CAUSAL && (j == i);
@@ -246,9 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->dp_free);
         const float2 nd2 = make_float2(nd, nd), sc2 = make_float2(scale, scale);
+        const float2 dps = make_float2(args.dp_scale, args.dp_scale);
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-          const float2 dpm = fadd2(make_float2(__uint_as_float(rr[2 * t]), __uint_as_float(rr[2 * t + 1])), nd2);
+          const float2 dpm = ffma2(make_float2(__uint_as_float(rr[2 * t]), __uint_as_float(rr[2 * t + 1])), dps, nd2);
           const float2 ds = fmul2(fmul2(make_float2(p[2 * t], p[2 * t + 1]), sc2), dpm);
           w[t] = pack_bf16x2(ds.x, ds.y);
         }

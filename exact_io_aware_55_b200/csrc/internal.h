@@ -90,10 +90,18 @@ struct BwdArgs {
   int N;
   int Np;             // N rounded up to a multiple of 128
   int BH;
-  float c_log2;       // scale * log2(e)
-  float scale;
+  float c_log2;       // scale * log2(e) (times the q and k descales for e4m3 inputs)
+  float dp_scale;     // factor on dP = dO V^T as computed (1, or the v descale for e4m3 inputs)
+  float dk_scale;     // dK = dk_scale * dS^T Q as computed (scale, or scale * q descale)
+  float dq_scale;     // dQ = dq_scale * dS K as computed (scale, or scale * k descale)
   int head_group;     // causal: heads per ordering group (see causal_block_order)
 };
+
+// Exact widening of e4m3 bytes to bf16 (every e4m3 value is a bf16 value):
+// `n16` groups of 16 elements from `src` to `dst`, grid-stride.  Used by the
+// backward of the e4m3 forward to give the bf16 backward kernels the very
+// values the forward multiplied.
+cudaError_t launch_widen_e4m3(const void* src, void* dst, long long n16, cudaStream_t stream);
 
 // Causal grids are one-dimensional: n_units work units (query-tile pairs,
 // key tiles, query tiles) per head, whose cost grows or shrinks linearly with

@@ -174,6 +174,38 @@ FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, floa
                      void* stream);
 
 /*
+ * Backward pass of fa_fwd_fp8: gradients with respect to the real inputs
+ * q8 * q_descale, k8 * k_descale, v8 * v_descale of the e4m3 forward
+ * ("What changed between FlashAttention 1, 2, and 3?" names low-precision
+ * FP8 as the forward's speed lever; the backward is the chain rule of the same
+ * attention, as in fa_bwd).
+ * Every e4m3 value is exactly a bf16 value, so the e4m3 Q, K and V are first
+ * widened to bf16 in the workspace (no rounding) and the bf16 backward
+ * kernels run on them; the descales are folded into the score factor
+ * (scale * q_descale * k_descale), into dP (v_descale), dK (scale * q_descale)
+ * and dQ (scale * k_descale).  The probabilities P and the gradient dS stay
+ * bf16: normalised P is about 1/N (below e4m3's smallest subnormal, 2^-9, at
+ * N >= 1024 with diffuse attention) and dS has a data-dependent range, so
+ * neither fits a per-tensor e4m3 scale.
+ *   q8, k8, v8 : in,  e4m3 (fn) bytes [B,H,N,d] (the forward's inputs)
+ *   o          : in,  bf16 [B,H,N,d] (fa_fwd_fp8's output)
+ *   dO         : in,  bf16 [B,H,N,d]
+ *   lse        : in,  fp32 [B,H,N] (fa_fwd_fp8's LSE)
+ *   dq, dk, dv : out, bf16 [B,H,N,d], in the real (descaled) units
+ *   workspace  : >= fa_bwd_fp8_workspace_size(B,H,N,d) bytes (fa_bwd's
+ *                workspace plus the three widened tensors, 6 N d bytes per head)
+ * d must be 128 (as fa_fwd_fp8); causal is supported; descales must be
+ * finite and > 0.  dQ is reduced with fp32 atomics as in fa_bwd.
+ */
+FA_API fa_status fa_bwd_fp8(const void* q8, const void* k8, const void* v8, float q_descale, float k_descale,
+                            float v_descale, const void* o, const void* dO, const float* lse, void* dq, void* dk,
+                            void* dv, int B, int H, int N, int d, float scale, int causal, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace fa_bwd_fp8 needs ((size_t)-1 for invalid arguments or d != 128). */
+FA_API size_t fa_bwd_fp8_workspace_size(int B, int H, int N, int d);
+
+/*
  * Backward pass for callers that cannot allocate device memory.  The pages
  * have no counterpart: this is a packaging variant of fa_bwd, not a step of
  * the method.  Some callers cannot call cudaMalloc where they run the

@@ -32,12 +32,23 @@ def _eval(expr: str, extra=None) -> int:
     return int(eval(expr, {"__builtins__": {}}, env))  # noqa: S307 -- arithmetic on known names only
 
 
+def _literal_constants(src: str) -> dict[str, int]:
+    """`constexpr int NAME = <integer literal>;` definitions of a source file."""
+    return {m.group(1): int(m.group(2)) for m in re.finditer(r"constexpr int (\w+)\s*=\s*(\d+)\s*;", src)}
+
+
 def barrier_counts(name: str) -> dict[str, int]:
-    """{barrier: arrive count} from every `mbar_init(&<obj>-><barrier>[...], count)`
+    """{barrier: arrive count} from every `mbar_init(&<obj>-><barrier>[...]..., count)`
     in the source file (array barriers share one count; the last init wins)."""
+    src = _source(name)
+    env = {}
+    for inc in re.findall(r'#include "([\w.]+)"', src):   # constants of the file's own headers
+        if os.path.exists(os.path.join(CSRC, inc)):
+            env.update(_literal_constants(_source(inc)))
+    env.update(_literal_constants(src))
     out = {}
-    for m in re.finditer(r"mbar_init\(&\w+->(\w+)(?:\[[^\]]*\])?,\s*([^;]+?)\);", _source(name)):
-        out[m.group(1)] = _eval(m.group(2))
+    for m in re.finditer(r"mbar_init\(&\w+->(\w+)(?:\[[^\]]*\])*,\s*([^;]+?)\);", src):
+        out[m.group(1)] = _eval(m.group(2), env)
     if not out:
         raise ValueError(f"no mbar_init found in {name}")
     return out

@@ -207,3 +207,22 @@ def test_get_device_status_without_a_gpu():
     if fa.lib.fa_get_device_status(None) == C["FA_OK"]:
         pytest.skip("a GPU is visible")
     assert fa.lib.fa_get_device_status(None) == C["FA_ERR_ARCH"]
+
+
+def test_fp8_backward_argument_errors_launch_nothing():
+    p = 4096
+    need = fa.fa_bwd_fp8_workspace_size(1, 1, 64, 128)
+    assert need > fa.fa_bwd_workspace_size(1, 1, 64, 128)
+    # bf16 workspace + three widened [BH, N, d] bf16 tensors
+    base = (fa.fa_bwd_workspace_size(1, 1, 64, 128) + 255) // 256 * 256
+    assert need == base + 2 * ((64 * 128 * 2 + 255) // 256 * 256) + 64 * 128 * 2
+    assert fa.lib.fa_bwd_fp8_workspace_size(1, 1, 64, 64) == ctypes.c_size_t(-1).value
+
+    def call(d=128, qd=1.0, ws=need, N=64):
+        return fa.lib.fa_bwd_fp8(p, p, p, F(qd), F(1.0), F(1.0), p, p, p, p, p, p, 1, 1, N, d, F(0.125), 0,
+                                 p, ws, None)
+    assert call(d=64) == C["FA_ERR_UNSUPPORTED"]
+    assert call(qd=0.0) == C["FA_ERR_INVALID_ARG"]
+    assert call(qd=float("nan")) == C["FA_ERR_INVALID_ARG"]
+    assert call(ws=need - 1) == C["FA_ERR_WORKSPACE"]
+    assert call(N=0) == C["FA_OK"]
