@@ -326,18 +326,23 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
-    # the dominant kernel: the backward's recompute kernel, 2.5 F of this rank's slice per launch
+    # The dominant kernel: the backward's recompute kernel, 2.5 F of this rank's
+    # slice per launch.  It is timed inside a long step (K steps of fwd + bwd
+    # back to back, seconds under the 1 kW power cap), so its denominator is the
+    # sustained bf16 figure; the burst one is reported beside it.
     main_tflops = 2.5 * F_rank / (t_main * 1e-3) / 1e12 if nh else 0.0
     call_tflops = 2.5 * F_rank / (t_bwd * 1e-3) / 1e12 if nh else 0.0
     roof = {"bound": "tensor", "kernel": "bwd_kernel<128, causal> (the backward's recompute kernel)",
-            "achieved": round(main_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(main_tflops / peak, 4),
+            "achieved": round(main_tflops, 2), "peak": peak_sus, "unit": "TFLOP/s",
+            "frac": round(main_tflops / peak_sus, 4),
             "traffic": committed_traffic("bwd_kernel", WORKLOAD_NAME) if ws == 1 else None,
             "algorithmic_flops_per_launch": 2.5 * F_rank,
             "ms_per_launch": round(t_main, 5),
-            "peak_source": f"{peak_src} bf16_tflops (burst)",
-            "frac_of_sustained_peak": round(main_tflops / peak_sus, 4),
-            "fa_bwd_call": {"achieved": round(call_tflops, 2), "frac": round(call_tflops / peak, 4),
+            "peak_source": f"{peak_src} bf16_tflops_sustained (the kernel runs inside a seconds-long loaded "
+                           f"region; see clocks)",
+            "peak_burst": peak, "frac_of_burst_peak": round(main_tflops / peak, 4),
+            "fa_bwd_call": {"achieved": round(call_tflops, 2), "frac": round(call_tflops / peak_sus, 4),
+                            "frac_of_burst_peak": round(call_tflops / peak, 4),
                             "ms": round(t_bwd, 5), "ms_preprocess": round(t_pre, 5),
                             "ms_dq_convert": round(t_fin, 5)}}
 
