@@ -220,3 +220,46 @@ def test_fp8_bwd_rejects_d64_and_bad_descales():
         fa.fa_bwd_fp8(y8, y8, y8, 1.0, 1.0, 1.0, y, y, lse, *outs, 0.1, False, small)
     assert e.value.status == fa.STATUS_CODES["FA_ERR_WORKSPACE"]
     del x8
+
+
+@pytest.mark.parametrize("mult", [8.0, 64.0])
+def test_fp8_large_score_range(mult):
+    """Q scaled by a power of two before quantisation: peaked rows and frequent
+    running-max moves.  The e4m3 forward takes its exponentials in half
+    precision, so LSE is checked here at 1e-3 where the largest terms dominate
+    the row sum."""
+    inp = synth.attention_inputs(1, 2, 1024, 128, seed=77, q_mult=mult, storage="e4m3")
+    for causal in (False, True):
+        o, lse, scale = _run(inp, causal)
+        o_ref, lse_ref = oracle.attention_forward(inp["q"], inp["k"], inp["v"], scale, causal)
+        _check(o, lse, o_ref, lse_ref, f"mult={mult} causal={causal}")
+
+
+def test_fp8_causal_forward_and_backward_b2_h16_n8192_d128_sampled():
+    """Causal e4m3 forward and its backward at B2 H16 N8192: sampled rows of O
+    and LSE, sampled dQ rows and dK/dV columns of two heads, and the gradient
+    sum identities on all 32 heads."""
+    B, H, N, d = 2, 16, 8192, 128
+    inp = synth.attention_inputs(B, H, N, d, seed=1253, storage="e4m3", want_f64=False)
+    do_bits = synth.to_bf16_bits(synth.normal_f32(1253, synth.TENSOR_IDS["do"], (B, H, N, d)))
+    q8, k8, v8 = (gu.dev_u8(inp[n + "_bits"]) for n in ("q", "k", "v"))
+    o, lse = fa.attention_forward_fp8(q8, k8, v8, inp["q_descale"], inp["k_descale"], inp["v_descale"], causal=True)
+    (dq, dk, dv), scale = _run_bwd_fp8(inp, do_bits, o, lse, True)
+    o64, lse64 = gu.to_f64(o), gu.to_f64(lse)
+    do_sum = np.stack([synth.bf16_bits_to_f64(do_bits[b, h]).sum(axis=0) for b in range(B) for h in range(H)])
+    dk_sum = dk.sum(axis=2).reshape(B * H, d)
+    dv_sum = dv.sum(axis=2).reshape(B * H, d)
+    assert np.max(np.abs(dk_sum) / np.linalg.norm(dk.reshape(B * H, -1), axis=1)[:, None]) <= 1e-2
+    assert np.max(np.abs(dv_sum - do_sum) / np.linalg.norm(do_sum, axis=1)[:, None]) <= 1e-2
+    for (b, h) in ((0, 0), (1, 15)):
+        rows = gu.sample_rows(N, 12, 5 + b * 16 + h)
+        cols = gu.sample_rows(N, 12, 6 + b * 16 + h)
+        qh, kh, vh = (synth.head_f64(inp, n, b, h) for n in ("q", "k", "v"))
+        doh = synth.bf16_bits_to_f64(do_bits[b, h])
+        o_ref, lse_ref = oracle.head_forward(qh, kh, vh, scale, True, rows=rows)
+        _check(o64[b, h][rows], lse64[b, h][rows], o_ref, lse_ref, f"head ({b},{h})")
+        rq, rk, rv = oracle.head_backward_sampled(qh, kh, vh, doh, scale, True, rows, cols)
+        for name, g, r, tol in zip(("dQ", "dK", "dV"), (dq[b, h][rows], dk[b, h][cols], dv[b, h][cols]),
+                                   (rq, rk, rv), (gu.FP8_O_REL_FRO, gu.FP8_O_REL_FRO, gu.GRAD_REL_FRO)):
+            e = gu.rel_fro(g, r)
+            assert e <= tol, f"{name} rel-Frobenius {e:.3e} head ({b},{h})"
