@@ -225,7 +225,11 @@ def run_ours(args):
             flush.fill_(1.0)                     # L2 flush, outside the events
             ev[i][0].record(stream)
             fa.fa_fwd(q, k, v, o, lse, scale, causal, stream)
-            fa.fa_bwd_events(q, k, v, o, do, lse, dq, dk, dv, scale, causal, work, ev[i][1:], stream)
+            if nh > 0:
+                fa.fa_bwd_events(q, k, v, o, do, lse, dq, dk, dv, scale, causal, work, ev[i][1:], stream)
+            else:                                # more ranks than heads: this rank has nothing to do
+                for e in ev[i][1:]:
+                    e.record(stream)
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
