@@ -49,6 +49,12 @@ L2_FLUSH_BYTES = 256 << 20
 BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
+def workload_config():
+    """The `config` of both arms' lines: the workload, its shape and its seed."""
+    return {"workload": WORKLOAD_NAME, **WORKLOAD, "seed": WORKLOAD_SEED, "global_batch": WORKLOAD["B"],
+            "seq_len": WORKLOAD["N"]}
+
+
 def fwd_flops(B, H, N, d, causal):
     f = 4.0 * B * H * N * N * d
     return f / 2.0 if causal else f
@@ -357,11 +363,10 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": round(t_step, 5), "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) Philox, rounded to bf16)",
-            "config": {"workload": WORKLOAD_NAME, "B": B, "H": H, "N": N, "d": d, "causal": causal,
-                       "seed": WORKLOAD_SEED, "global_batch": B, "seq_len": N,
-                       "parallelism": f"heads split over {ws} GPU(s), {nh} on rank 0, no data-path collective",
-                       "l2": "inputs (4 x 256 MiB per GPU at one GPU) exceed L2; plus a 256 MiB flush write "
-                             "between steps, outside the per-step CUDA events"},
+            "config": workload_config(),
+            "parallelism": f"heads split over {ws} GPU(s), {nh} on rank 0, no data-path collective",
+            "l2": "inputs (4 x 256 MiB at one GPU) exceed L2; plus a 256 MiB flush write between steps, "
+                  "outside the per-step CUDA events",
             "fwd_tflops": round(fwd_tflops, 2), "bwd_tflops": round(bwd_tflops, 2),
             "fwd_frac_of_peak": round(fwd_tflops / ws / peak, 4),
             "bwd_frac_of_peak": round(bwd_tflops / ws / peak, 4),
@@ -673,7 +678,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / max(1, args.steps),
         "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) Philox, rounded to bf16, evaluated in fp64)",
-        "config": {"workload": WORKLOAD_NAME, **WORKLOAD},
+        "config": workload_config(),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"each step: units of one head cut to its first {n} queries and keys "
                                    f"(fwd+bwd) for {args.ref_step_budget:.1f} s; {units_total} units in total"},
