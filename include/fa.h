@@ -39,6 +39,13 @@
  *     that runs out records a status readable with fa_device_status().
  *   - Thread safety: calls are re-entrant; the first call on a device also
  *     configures the kernels' shared-memory limits for that device.
+ *   - CUDA graphs: the attention calls (fa_fwd*, fa_bwd*, fa_fwd_decode,
+ *     fa_fwd_standard) only enqueue kernel launches on the stream, so a
+ *     caller may capture them into a graph and replay it.  Make the first
+ *     call on each device outside any capture (it looks up device attributes
+ *     and symbol addresses once).  fa_bwd_events also records the caller's
+ *     events, which time nothing inside a capture; fa_device_status
+ *     synchronises and cannot be captured.
  */
 #ifndef FA_H_
 #define FA_H_
