@@ -391,8 +391,9 @@ def run_ours(args):
 def run_case(args):
     """One named path on --shape, for profiling (a short JSON line, not the
     bench line): 'decode' (B,H,Nk,d with --nq queries, causal), 'standard'
-    (B,H,N,d: the materialising baseline, then the fused forward, per step) or
-    'fp8' (B,H,N,d: the e4m3 forward)."""
+    (B,H,N,d: the materialising baseline, then the fused forward, per step),
+    'fp8' (B,H,N,d: the e4m3 forward) or 'det' (B,H,N,d: the backward with the
+    deterministic dQ pass, after one forward)."""
     import torch
 
     import exact_io_aware_55_b200 as fa
@@ -418,6 +419,17 @@ def run_case(args):
         def step():
             fa.fa_fwd_decode(q, k, v, o, lse, d ** -0.5, True, work, stream)
         nbytes = 4 * B * H * N * d
+    elif args.case == "det":
+        q, k, v, do = rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), device=dev)
+        fa.fa_fwd(q, k, v, o, lse, d ** -0.5, args.causal, stream)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        work = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+
+        def step():
+            fa.fa_bwd_deterministic(q, k, v, o, do, lse, dq, dk, dv, d ** -0.5, args.causal, work, stream)
+        flops = 2.5 * fwd_flops(B, H, N, d, args.causal)
     elif args.case == "fp8":
         q8, k8, v8 = (torch.randn((B, H, N, d), generator=g, device=dev).mul_(100.0).clamp_(-448, 448)
                       .to(torch.float8_e4m3fn) for _ in range(3))
@@ -700,7 +712,7 @@ def main():
     ap.add_argument("--shape", default="", help="B,H,N,d of another workload (default: the bench workload)")
     ap.add_argument("--causal", action="store_true")
     ap.add_argument("--noncausal", action="store_true")
-    ap.add_argument("--case", choices=["decode", "standard", "fp8"], default="",
+    ap.add_argument("--case", choices=["decode", "standard", "fp8", "det"], default="",
                     help="profile one path on --shape instead of the bench step")
     ap.add_argument("--nq", type=int, default=1, help="queries per head for --case decode")
     ap.add_argument("--clock-window", type=float, default=1.5,
