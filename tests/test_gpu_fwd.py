@@ -101,6 +101,21 @@ def test_fwd_config_b2_h16_n8192_d128_causal_sampled(q_mult):
     _sampled_check(2, 16, 8192, 128, True, seed=1237, q_mult=q_mult)
 
 
+def test_fwd_config_b2_h16_n8192_d128_causal_q8_every_head():
+    """The large-score-range run of the causal B2 H16 N8192 d128 configuration
+    (Q x 8) against the oracle on every element of every head, not a sample:
+    with a peaked softmax, O sits next to single V rows, so this is where the
+    O max-abs bound is tightest (about 30 s of oracle time)."""
+    B, H, N, d = 2, 16, 8192, 128
+    inp = synth.attention_inputs(B, H, N, d, seed=1237, q_mult=8.0, with_grad=False, want_f64=False)
+    o, lse, scale = _run_fwd(inp, True)
+    for b in range(B):
+        for h in range(H):
+            qh, kh, vh = (synth.head_f64(inp, n, b, h) for n in ("q", "k", "v"))
+            o_ref, lse_ref = oracle.head_forward(qh, kh, vh, scale, True)
+            gu.assert_o_lse(o[b, h], lse[b, h], o_ref, lse_ref, f"head ({b},{h})")
+
+
 def test_fwd_config_b1_h32_n32768_d128_causal_sampled():
     _sampled_check(1, 32, 32768, 128, True, seed=1238, n_heads=2, n_rows=16)
 
