@@ -178,3 +178,58 @@ def test_bwd_events_matches_fa_bwd_and_orders_its_events(d, causal):
     parts = [ev[i].elapsed_time(ev[i + 1]) for i in range(3)]
     assert all(p >= 0.0 for p in parts) and parts[1] > 0.0
     assert fa.fa_device_status() == (0, 0)
+
+
+def _bf16_round(x):
+    """Round float64 values to bf16 (through float32, round to nearest even)."""
+    b = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16
+    return b.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def _bf16_rounding_reference(inp, o_dev, lse_dev, scale, causal):
+    """The backward's definition with P and dS rounded to bf16 where the
+    kernels round them (P for dV; dS, formed from the unrounded P, for dQ and
+    dK), from the device's own O and LSE.  Test-only: it pins where the device
+    path rounds, on problems where the fp64 result is not well conditioned."""
+    q, k, v, do = (inp[n] for n in ("q", "k", "v", "do"))
+    B, H, N, d = q.shape
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    for b in range(B):
+        for h in range(H):
+            s = scale * q[b, h] @ k[b, h].T
+            if causal:
+                s = np.where(np.tril(np.ones((N, N), bool)), s, -np.inf)
+            p = np.exp(s - lse_dev[b, h][:, None])
+            dvec = (do[b, h] * o_dev[b, h]).sum(1, keepdims=True)
+            dv[b, h] = _bf16_round(p).T @ do[b, h]
+            ds = _bf16_round(p * (do[b, h] @ v[b, h].T - dvec))
+            dq[b, h] = scale * ds @ k[b, h]
+            dk[b, h] = scale * ds.T @ q[b, h]
+    return dq, dk, dv
+
+
+# Tiny, peaked problems (from a seeded random sweep) where dP - D cancels: the
+# gradients were 1.1e-2 to 3.4e-2 from the fp64 oracle, all of it the bf16
+# rounding of dS, which every bf16 implementation of the method performs.
+TINY_PEAKED = [(2, 1, 4, 64, False, 8.0, 986825433), (1, 1, 2, 128, True, 1.0, 87362969),
+               (1, 1, 8, 128, False, 8.0, 714526692)]
+
+
+@pytest.mark.parametrize("deterministic", [False, True])
+@pytest.mark.parametrize("case", TINY_PEAKED)
+def test_bwd_tiny_peaked_matches_bf16_rounding_reference(case, deterministic):
+    B, H, N, d, causal, mult, seed = case
+    inp = synth.attention_inputs(B, H, N, d, seed=seed, q_mult=mult)
+    q, k, v, do = _device_inputs(inp)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = fa.attention_forward(q, k, v, scale=scale, causal=causal)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    work = torch.empty(max(16, fa.fa_bwd_workspace_size(B, H, N, d)), dtype=torch.uint8, device="cuda")
+    (fa.fa_bwd_deterministic if deterministic else fa.fa_bwd)(q, k, v, o, do, lse, dq, dk, dv, scale, causal, work)
+    torch.cuda.synchronize()
+    ref = _bf16_rounding_reference(inp, gu.to_f64(o), gu.to_f64(lse), scale, causal)
+    for name, g, r in zip(("dQ", "dK", "dV"), (dq, dk, dv), ref):
+        e = gu.rel_fro(gu.to_f64(g), r)
+        assert e <= 5e-3, f"{name} {e:.3e} against the bf16-rounding reference {case}"
+    assert fa.fa_device_status() == (0, 0)
